@@ -1,0 +1,195 @@
+/*
+ * mixq.h -- C ABI of libmixq.so, the B200 (sm_100a) outlier-decomposed
+ * mixed-precision quantized linear layer.
+ *
+ * The layer (MixQ article "一键部署LLM混合精度推理，端到端吞吐比AWQ最大提升6倍！",
+ * 研究背景 Fig. 5 and MixQ的解决方案 Figs. 10-12) splits Y = X W^T into
+ *   Y = diag(s_x) (Xq Wq^T) diag(s_w) + X_out W_out^T
+ * where Xq/Wq are INT8 codes of the dense part, and X_out/W_out hold the few
+ * fixed outlier channels, concatenated in their original order, in FP16.  The
+ * W4A8 variant (QServe W4A8KV4 reading notes, 渐进量化 / 寄存器压力和并行性;
+ * MixLLM page, "MixLLM: Ein neuer Ansatz") stores Wq as 4-bit group codes and
+ * expands them back to INT8 inside the GEMM mainloop, so every product still
+ * runs on INT8 tensor cores.
+ *
+ * Conventions for every call:
+ *   - All matrix pointers are DEVICE pointers owned by the caller; the library
+ *     allocates no device memory, keeps no state between calls (beyond cached
+ *     device attributes and a thread-local error string) and needs no
+ *     workspace.  Matrix pointers must be 16-byte aligned.
+ *   - fp16 data is IEEE binary16, passed as void*.  Matrices are row-major.
+ *   - Every call is asynchronous on `stream` (a cudaStream_t passed as void*;
+ *     NULL = the legacy default stream).  Errors a host can see (bad sizes,
+ *     null or misaligned pointers, no device) return synchronously as a
+ *     mixq_status and leave the stream untouched.  Errors only the device can
+ *     see (an invalid outlier list, a wait that ran out of time) are written
+ *     to `*status` (a device int32 the caller zeroes; the first error wins;
+ *     may be NULL to ignore them); read it after synchronizing the stream.
+ *   - mixq_last_error() returns a thread-local description of the last
+ *     non-OK status returned on the calling thread.
+ *   - Calls that share output buffers must not overlap on the GPU.
+ *
+ * Shape rules (MIXQ_ERR_UNSUPPORTED_SHAPE otherwise): K % 128 == 0, K > 0,
+ * N % 128 == 0, N > 0, M >= 0, 0 <= K_out <= K.  K_out_pad is K_out rounded up
+ * to a multiple of 64; the padding columns of X_out / W_out are zero-filled by
+ * the library.
+ */
+#ifndef MIXQ_H
+#define MIXQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mixq_status {
+  MIXQ_OK = 0,
+  MIXQ_ERR_INVALID_ARG = 1,      /* null pointer, bad leading dimension, bad mode, bad idx */
+  MIXQ_ERR_UNSUPPORTED_SHAPE = 2,/* violates the shape rules above */
+  MIXQ_ERR_MISALIGNED = 3,       /* a matrix pointer or row pitch is not 16-byte aligned */
+  MIXQ_ERR_CUDA = 4,             /* a CUDA runtime/driver call failed (see mixq_last_error) */
+  MIXQ_ERR_TIMEOUT = 5,          /* device only: a pipeline wait ran out of time */
+  MIXQ_ERR_NO_DEVICE = 6         /* no usable sm_100 device is current */
+} mixq_status;
+
+/* Weight formats. */
+enum { MIXQ_W8 = 0, MIXQ_W4G128 = 1 };
+
+/* Thread-local text for the last non-OK status returned on this thread. */
+const char *mixq_last_error(void);
+
+/* ABI version (major*100 + minor). */
+int mixq_version(void);
+
+/*
+ * Sizes of the prepacked weight buffers for mode, N, K, K_out (host only).
+ *   *wq_bytes   MIXQ_W8: N*K (int8 codes, row-major [N][K]).
+ *               MIXQ_W4G128: N*K/2 (two 4-bit codes per byte, see below).
+ *   *grp_bytes  MIXQ_W4G128: 4*N*(K/128) (one fp16 pair (s2, z2) per group,
+ *               group-major [K/128][N]); MIXQ_W8: 0.
+ *   *wout_bytes 2*N*K_out_pad (fp16 [N][K_out_pad]).
+ * Any output pointer may be NULL.
+ */
+mixq_status mixq_prepack_size(int mode, int N, int K, int K_out, size_t *wq_bytes,
+                              size_t *grp_bytes, size_t *wout_bytes);
+
+/*
+ * Offline weight prepack (MixQ Fig. 5: weights in low bits; Fig. 11: outlier
+ * columns extracted in original order; QServe 渐进量化 + group-wise: 4-bit level).
+ *   W      fp16 [N][K]           input weights (read only)
+ *   idx    int32 [K_out]          outlier channels, sorted ascending, unique,
+ *                                 inside [0, K) (checked on the device)
+ *   Wq     MIXQ_W8: int8 [N][K], code = clamp(rint(W * 127/a), -127, 127) with
+ *          a = max_k |W[n,k]| over all K; MIXQ_W4G128: packed level-2 codes,
+ *          byte (n, g*64 + b) holds q[n, 128g + 8(b>>2) + (b&3)] in its low
+ *          nibble and q[n, same + 4] in its high nibble.
+ *   s_w    fp32 [N]               a / 127
+ *   grp    MIXQ_W4G128 only (else NULL): fp16 pairs (s2, z2) at [g][n], with
+ *          s2 = max(1, ceil((hi-lo)/15)), z2 = clamp(rint(-lo/s2), 0, 15) over
+ *          the group's INT8 codes, q = clamp(rint(w8/s2)+z2, qlo, qhi) so the
+ *          effective weight (q - z2)*s2 always fits int8.
+ *   W_out  fp16 [N][K_out_pad]    W[:, idx[j]] for j < K_out, zero after; may be
+ *                                 NULL when K_out == 0.
+ */
+mixq_status mixq_prepack_weights(int mode, const void *W, int N, int K, const int32_t *idx,
+                                 int K_out, void *Wq, float *s_w, void *grp, void *W_out,
+                                 int32_t *status, void *stream);
+
+/*
+ * Fused amax + threshold test + outlier gather + INT8 quantization of the
+ * activations (MixQ MixQ的解决方案: the amax taken for quantization shows
+ * whether outliers exist; Fig. 10 equivalent transformation; Fig. 11 order-
+ * preserved outlier matrix).  Per token m:
+ *   aI = max_{k in idx} |x|, aN = max_{k not in idx} |x|
+ *   mixed = K_out > 0 && max(aI, aN) > threshold        (strictly greater)
+ *   a = mixed ? aN : max(aI, aN),  s_x[m] = a / 127
+ *   Xq[m,k] = (mixed && k in idx) ? 0 : clamp(rint(x * 127/a), -127, 127)
+ *   X_out[m,j] = (mixed && j < K_out) ? X[m, idx[j]] : 0
+ *   X              fp16 [M][ldx], ldx >= K, ldx % 8 == 0 (read only)
+ *   Xq             int8 [M][K]
+ *   s_x            fp32 [M]
+ *   X_out          fp16 [M][K_out_pad] (may be NULL when K_out == 0)
+ *   detect_bitmap  uint32 [ceil(K/32)]: bit k%32 of word k/32 is set iff some
+ *                  token has |X[m,k]| > threshold (written, not accumulated)
+ *   flags          int32 [4]: [0] = number of mixed tokens, [1] = number of
+ *                  detected channels that are not in idx, [2] and [3] are used
+ *                  by the call and read 0 when it completes.  gemm calls read
+ *                  flags[0] on the device to skip the FP16 slice when no
+ *                  token is mixed.
+ * Launches two kernels (a 1-block reset of bitmap/flags, then the main pass).
+ */
+mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx, int K_out,
+                              float threshold, int8_t *Xq, float *s_x, void *X_out,
+                              uint32_t *detect_bitmap, int32_t *flags, int32_t *status,
+                              void *stream);
+
+/*
+ * Mixed-precision GEMM, 8-bit weights (MixQ Fig. 5 decomposition; Fig. 12
+ * fused dequantize, scale and add of the INT32 result in registers):
+ *   acc[m,n] = sum_k Xq[m,k] Wq[n,k]                     (exact INT32, tcgen05 kind::i8)
+ *   o[m,n]   = sum_j X_out[m,j] W_out[n,j]               (fp32, tcgen05 kind::f16;
+ *                                                         skipped if flags[0] == 0)
+ *   Y[m,n]   = fp16((float(acc) * s_x[m]) * s_w[n] + o)
+ *   Xq int8 [M][K], s_x fp32 [M], X_out fp16 [M][K_out_pad] (NULL if K_out == 0),
+ *   Wq/s_w/W_out from mixq_prepack_weights(MIXQ_W8), flags int32 [4] from
+ *   mixq_quantize_act (NULL means "some token may be mixed"),
+ *   Y fp16 [M][ldy], ldy >= N, ldy % 8 == 0.
+ */
+mixq_status mixq_gemm_w8a8o16(int M, int N, int K, int K_out, const int8_t *Xq, const float *s_x,
+                              const void *X_out, const void *Wq, const float *s_w,
+                              const void *W_out, const int32_t *flags, void *Y, int ldy,
+                              int32_t *status, void *stream);
+
+/*
+ * Same layer with 4-bit group-wise weights (QServe 渐进量化 / 寄存器压力和并行性,
+ * MixLLM two-stage dequantization): inside the mainloop every 4-bit code is
+ * expanded back to the INT8 weight (q - z2)*s2, four codes per 32-bit
+ * register operation, and multiplied on INT8 tensor cores.
+ *   Wq4/grp/s_w/W_out from mixq_prepack_weights(MIXQ_W4G128); the rest as
+ *   mixq_gemm_w8a8o16.
+ */
+mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, const float *s_x,
+                              const void *X_out, const void *Wq4, const void *grp,
+                              const float *s_w, const void *W_out, const int32_t *flags, void *Y,
+                              int ldy, int32_t *status, void *stream);
+
+/*
+ * The launch plan the gemm calls use for a shape (host only, no GPU needed):
+ * output tile width *bn (128 or 256 columns; tiles are 128 rows high), the
+ * K-split factor *split (thread-block cluster size along K, 1..8) and the
+ * number of CTAs *ctas.  num_sms <= 0 means "query the current device".
+ */
+mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, int *split,
+                           int *ctas);
+
+/*
+ * Test-only: the gemm mainloop alone, raw INT32 accumulators out
+ * (acc int32 [M][ldacc]).  mode MIXQ_W8 uses Wq; MIXQ_W4G128 uses Wq4 + grp.
+ * bn/split override the plan when > 0.
+ */
+mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq, const void *Wq,
+                                const void *grp, int32_t *acc, int ldacc, int bn, int split,
+                                int32_t *status, void *stream);
+
+/* Test-only: logical 4-bit codes back from the packed layout:
+ * q uint8 [N][K], s2/z2 uint8 [N][K/128]. */
+mixq_status mixq_debug_unpack_w4(int N, int K, const void *Wq4, const void *grp, uint8_t *q,
+                                 uint8_t *s2, uint8_t *z2, int32_t *status, void *stream);
+
+/*
+ * Test-only: the W8 gemm kernel with its TMA producer told to issue nothing
+ * and every pipeline wait limited to wait_limit_ns.  The kernel must return
+ * on its own and write MIXQ_ERR_TIMEOUT to *status; used to check that a
+ * stalled pipeline ends with an error instead of hanging the GPU.
+ */
+mixq_status mixq_debug_gemm_stall(int M, int N, int K, const int8_t *Xq, const void *Wq,
+                                  const float *s_x, const float *s_w, void *Y, int ldy,
+                                  uint64_t wait_limit_ns, int32_t *status, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MIXQ_H */

@@ -1,0 +1,331 @@
+// extern "C" boundary of libmixq.so (declared and documented in include/mixq.h):
+// argument validation that the host can do, device checks, dispatch to the
+// kernel launchers, and the thread-local error text.
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <string>
+
+#include "../../include/mixq.h"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error = "no error";
+
+mixq_status fail(mixq_status s, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+mixq_status ok() { return MIXQ_OK; }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;  // 2 s per pipeline wait
+
+// Device checks: a current device with compute capability 10.x.
+mixq_status check_device(int *sms) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return fail(MIXQ_ERR_NO_DEVICE, "no CUDA device is available");
+  }
+  if (mixq::device_cc_major(dev) != 10)
+    return fail(MIXQ_ERR_NO_DEVICE, "device %d is not an sm_100 (Blackwell B200-class) GPU", dev);
+  if (sms) *sms = mixq::device_sm_count(dev);
+  return MIXQ_OK;
+}
+
+mixq_status from_cuda(cudaError_t e, const char *what, const char *why = nullptr) {
+  if (e == cudaSuccess) return MIXQ_OK;
+  return fail(MIXQ_ERR_CUDA, "%s: %s%s%s", what, cudaGetErrorString(e), why ? " -- " : "",
+              why ? why : "");
+}
+
+mixq_status check_shape(int M, int N, int K, int K_out) {
+  if (M < 0) return fail(MIXQ_ERR_UNSUPPORTED_SHAPE, "M = %d must be >= 0", M);
+  if (N <= 0 || N % 128) return fail(MIXQ_ERR_UNSUPPORTED_SHAPE, "N = %d must be a positive multiple of 128", N);
+  if (K <= 0 || K % 128) return fail(MIXQ_ERR_UNSUPPORTED_SHAPE, "K = %d must be a positive multiple of 128", K);
+  if (K_out < 0 || K_out > K)
+    return fail(MIXQ_ERR_UNSUPPORTED_SHAPE, "K_out = %d must lie in [0, K = %d]", K_out, K);
+  return MIXQ_OK;
+}
+
+}  // namespace
+
+namespace mixq {
+
+namespace {
+struct DevAttr {
+  std::atomic<int> sms{0};
+  std::atomic<int> major{-1};
+  std::atomic<long long> smem{0};
+};
+DevAttr g_attr[64];
+
+void fill_attr(int dev) {
+  if (dev < 0 || dev >= 64) return;
+  if (g_attr[dev].major.load() >= 0) return;
+  int sms = 0, major = 0, smem = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&smem, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev);
+  g_attr[dev].sms = sms;
+  g_attr[dev].smem = smem;
+  g_attr[dev].major = major;
+}
+}  // namespace
+
+int device_sm_count(int dev) {
+  fill_attr(dev);
+  return dev >= 0 && dev < 64 ? g_attr[dev].sms.load() : 0;
+}
+int device_cc_major(int dev) {
+  fill_attr(dev);
+  return dev >= 0 && dev < 64 ? g_attr[dev].major.load() : 0;
+}
+size_t device_max_smem_optin(int dev) {
+  fill_attr(dev);
+  return dev >= 0 && dev < 64 ? static_cast<size_t>(g_attr[dev].smem.load()) : 0;
+}
+
+}  // namespace mixq
+
+extern "C" {
+
+const char *mixq_last_error(void) { return g_last_error.c_str(); }
+
+int mixq_version(void) { return 100; }
+
+mixq_status mixq_prepack_size(int mode, int N, int K, int K_out, size_t *wq_bytes,
+                              size_t *grp_bytes, size_t *wout_bytes) {
+  if (mode != MIXQ_W8 && mode != MIXQ_W4G128) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
+  mixq_status s = check_shape(0, N, K, K_out);
+  if (s != MIXQ_OK) return s;
+  const size_t n = static_cast<size_t>(N), k = static_cast<size_t>(K);
+  if (wq_bytes) *wq_bytes = mode == MIXQ_W8 ? n * k : n * k / 2;
+  if (grp_bytes) *grp_bytes = mode == MIXQ_W8 ? 0 : 4 * n * (k / 128);
+  if (wout_bytes) *wout_bytes = 2 * n * static_cast<size_t>(mixq::k_out_pad(K_out));
+  return ok();
+}
+
+mixq_status mixq_prepack_weights(int mode, const void *W, int N, int K, const int32_t *idx,
+                                 int K_out, void *Wq, float *s_w, void *grp, void *W_out,
+                                 int32_t *status, void *stream) {
+  if (mode != MIXQ_W8 && mode != MIXQ_W4G128) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
+  mixq_status s = check_shape(0, N, K, K_out);
+  if (s != MIXQ_OK) return s;
+  if (!W || !Wq || !s_w) return fail(MIXQ_ERR_INVALID_ARG, "W, Wq and s_w must be non-null");
+  if (mode == MIXQ_W4G128 && !grp) return fail(MIXQ_ERR_INVALID_ARG, "grp must be non-null for MIXQ_W4G128");
+  if (K_out > 0 && (!idx || !W_out))
+    return fail(MIXQ_ERR_INVALID_ARG, "idx and W_out must be non-null when K_out > 0");
+  if (!aligned16(W) || !aligned16(Wq) || !aligned16(s_w) || (grp && !aligned16(grp)) ||
+      (W_out && !aligned16(W_out)))
+    return fail(MIXQ_ERR_MISALIGNED, "matrix pointers must be 16-byte aligned");
+  s = check_device(nullptr);
+  if (s != MIXQ_OK) return s;
+  return from_cuda(mixq::launch_prepack(mode, W, N, K, idx, K_out, Wq, s_w, grp, W_out, status,
+                                        static_cast<cudaStream_t>(stream)),
+                   "prepack launch");
+}
+
+mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx, int K_out,
+                              float threshold, int8_t *Xq, float *s_x, void *X_out,
+                              uint32_t *detect_bitmap, int32_t *flags, int32_t *status,
+                              void *stream) {
+  mixq_status s = check_shape(M, 128, K, K_out);
+  if (s != MIXQ_OK) return s;
+  if (ldx < K || ldx % 8) return fail(MIXQ_ERR_INVALID_ARG, "ldx = %d must be >= K and a multiple of 8", ldx);
+  if (!(threshold >= 0.f) || threshold != threshold)
+    return fail(MIXQ_ERR_INVALID_ARG, "threshold must be a finite value >= 0");
+  if (!detect_bitmap || !flags) return fail(MIXQ_ERR_INVALID_ARG, "detect_bitmap and flags must be non-null");
+  if (M > 0 && (!X || !Xq || !s_x)) return fail(MIXQ_ERR_INVALID_ARG, "X, Xq and s_x must be non-null");
+  if (K_out > 0 && !idx) return fail(MIXQ_ERR_INVALID_ARG, "idx must be non-null when K_out > 0");
+  if (K_out > 0 && M > 0 && !X_out) return fail(MIXQ_ERR_INVALID_ARG, "X_out must be non-null when K_out > 0");
+  if ((X && !aligned16(X)) || (Xq && !aligned16(Xq)) || (X_out && !aligned16(X_out)) ||
+      !aligned16(detect_bitmap) || !aligned16(flags))
+    return fail(MIXQ_ERR_MISALIGNED, "matrix pointers must be 16-byte aligned");
+  int sms = 0;
+  s = check_device(&sms);
+  if (s != MIXQ_OK) return s;
+  return from_cuda(mixq::launch_quantize_act(X, M, K, ldx, idx, K_out, threshold, Xq, s_x, X_out,
+                                             detect_bitmap, flags, status,
+                                             static_cast<cudaStream_t>(stream), sms),
+                   "quantize launch");
+}
+
+static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const int8_t *Xq,
+                               const float *s_x, const void *X_out, const void *Wq,
+                               const void *grp, const float *s_w, const void *W_out,
+                               const int32_t *flags, void *Y, int ldy, int32_t *status,
+                               void *stream) {
+  mixq_status s = check_shape(M, N, K, K_out);
+  if (s != MIXQ_OK) return s;
+  if (ldy < N || ldy % 8) return fail(MIXQ_ERR_INVALID_ARG, "ldy = %d must be >= N and a multiple of 8", ldy);
+  if (M == 0) return check_device(nullptr);
+  if (!Xq || !s_x || !Wq || !s_w || !Y)
+    return fail(MIXQ_ERR_INVALID_ARG, "Xq, s_x, Wq, s_w and Y must be non-null");
+  if (mode == MIXQ_W4G128 && !grp) return fail(MIXQ_ERR_INVALID_ARG, "grp must be non-null");
+  if (K_out > 0 && (!X_out || !W_out))
+    return fail(MIXQ_ERR_INVALID_ARG, "X_out and W_out must be non-null when K_out > 0");
+  if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(Y) || !aligned16(s_w) ||
+      (grp && !aligned16(grp)) || (X_out && !aligned16(X_out)) || (W_out && !aligned16(W_out)))
+    return fail(MIXQ_ERR_MISALIGNED, "matrix pointers must be 16-byte aligned");
+  int sms = 0;
+  s = check_device(&sms);
+  if (s != MIXQ_OK) return s;
+  mixq::GemmArgs a{};
+  a.mode = mode;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.K_out = K_out;
+  a.Xq = Xq;
+  a.s_x = s_x;
+  a.X_out = X_out;
+  a.Wq = Wq;
+  a.grp = grp;
+  a.s_w = s_w;
+  a.W_out = W_out;
+  a.flags = flags;
+  a.Y = Y;
+  a.ldy = ldy;
+  a.epi = mixq::Epi::kMixed;
+  a.status = status;
+  a.wait_limit_ns = kDefaultWaitNs;
+  const mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms);
+  const char *why = nullptr;
+  return from_cuda(mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why),
+                   "gemm launch", why);
+}
+
+mixq_status mixq_gemm_w8a8o16(int M, int N, int K, int K_out, const int8_t *Xq, const float *s_x,
+                              const void *X_out, const void *Wq, const float *s_w,
+                              const void *W_out, const int32_t *flags, void *Y, int ldy,
+                              int32_t *status, void *stream) {
+  return gemm_common(MIXQ_W8, M, N, K, K_out, Xq, s_x, X_out, Wq, nullptr, s_w, W_out, flags, Y,
+                     ldy, status, stream);
+}
+
+mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, const float *s_x,
+                              const void *X_out, const void *Wq4, const void *grp,
+                              const float *s_w, const void *W_out, const int32_t *flags, void *Y,
+                              int ldy, int32_t *status, void *stream) {
+  return gemm_common(MIXQ_W4G128, M, N, K, K_out, Xq, s_x, X_out, Wq4, grp, s_w, W_out, flags, Y,
+                     ldy, status, stream);
+}
+
+mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, int *split,
+                           int *ctas) {
+  if (mode != MIXQ_W8 && mode != MIXQ_W4G128) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
+  mixq_status s = check_shape(M, N, K, 0);
+  if (s != MIXQ_OK) return s;
+  if (num_sms <= 0) {
+    s = check_device(&num_sms);
+    if (s != MIXQ_OK) return s;
+  }
+  const mixq::GemmPlan p = mixq::plan_gemm(mode, M, N, K, num_sms);
+  if (bn) *bn = p.bn;
+  if (split) *split = p.split;
+  if (ctas) *ctas = p.ctas;
+  return ok();
+}
+
+mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq, const void *Wq,
+                                const void *grp, int32_t *acc, int ldacc, int bn, int split,
+                                int32_t *status, void *stream) {
+  if (mode != MIXQ_W8 && mode != MIXQ_W4G128) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
+  mixq_status s = check_shape(M, N, K, 0);
+  if (s != MIXQ_OK) return s;
+  if (ldacc < N || ldacc % 4) return fail(MIXQ_ERR_INVALID_ARG, "ldacc = %d must be >= N and a multiple of 4", ldacc);
+  if (bn != 0 && bn != 128 && bn != 256) return fail(MIXQ_ERR_INVALID_ARG, "bn = %d", bn);
+  if (split < 0 || split > 8)
+    return fail(MIXQ_ERR_INVALID_ARG, "split = %d", split);
+  if (split > K / 128) return fail(MIXQ_ERR_UNSUPPORTED_SHAPE, "split %d exceeds K/128", split);
+  if (M == 0) return check_device(nullptr);
+  if (!Xq || !Wq || !acc || (mode == MIXQ_W4G128 && !grp))
+    return fail(MIXQ_ERR_INVALID_ARG, "null pointer");
+  if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(acc) || (grp && !aligned16(grp)))
+    return fail(MIXQ_ERR_MISALIGNED, "matrix pointers must be 16-byte aligned");
+  int sms = 0;
+  s = check_device(&sms);
+  if (s != MIXQ_OK) return s;
+  mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms);
+  if (bn) plan.bn = bn;
+  if (split) plan.split = split;
+  mixq::GemmArgs a{};
+  a.mode = mode;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.Xq = Xq;
+  a.Wq = Wq;
+  a.grp = grp;
+  a.Y = acc;
+  a.ldy = ldacc;
+  a.epi = mixq::Epi::kRawI32;
+  a.status = status;
+  a.wait_limit_ns = kDefaultWaitNs;
+  const char *why = nullptr;
+  return from_cuda(mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why),
+                   "debug gemm launch", why);
+}
+
+mixq_status mixq_debug_unpack_w4(int N, int K, const void *Wq4, const void *grp, uint8_t *q,
+                                 uint8_t *s2, uint8_t *z2, int32_t *status, void *stream) {
+  (void)status;
+  mixq_status s = check_shape(0, N, K, 0);
+  if (s != MIXQ_OK) return s;
+  if (!Wq4 || !grp || !q || !s2 || !z2) return fail(MIXQ_ERR_INVALID_ARG, "null pointer");
+  s = check_device(nullptr);
+  if (s != MIXQ_OK) return s;
+  return from_cuda(mixq::launch_unpack_w4(N, K, Wq4, grp, q, s2, z2,
+                                          static_cast<cudaStream_t>(stream)),
+                   "unpack launch");
+}
+
+mixq_status mixq_debug_gemm_stall(int M, int N, int K, const int8_t *Xq, const void *Wq,
+                                  const float *s_x, const float *s_w, void *Y, int ldy,
+                                  uint64_t wait_limit_ns, int32_t *status, void *stream) {
+  mixq_status s = check_shape(M, N, K, 0);
+  if (s != MIXQ_OK) return s;
+  if (M == 0 || !Xq || !Wq || !s_x || !s_w || !Y || !status)
+    return fail(MIXQ_ERR_INVALID_ARG, "null pointer or M == 0");
+  if (ldy < N || ldy % 8) return fail(MIXQ_ERR_INVALID_ARG, "ldy");
+  if (wait_limit_ns == 0 || wait_limit_ns > kDefaultWaitNs)
+    return fail(MIXQ_ERR_INVALID_ARG, "wait_limit_ns must lie in (0, 2 s]");
+  int sms = 0;
+  s = check_device(&sms);
+  if (s != MIXQ_OK) return s;
+  mixq::GemmArgs a{};
+  a.mode = MIXQ_W8;
+  a.M = M;
+  a.N = N;
+  a.K = K;
+  a.Xq = Xq;
+  a.Wq = Wq;
+  a.s_x = s_x;
+  a.s_w = s_w;
+  a.Y = Y;
+  a.ldy = ldy;
+  a.epi = mixq::Epi::kMixed;
+  a.status = status;
+  a.wait_limit_ns = wait_limit_ns;
+  a.debug_stall = 1;
+  mixq::GemmPlan plan = mixq::plan_gemm(MIXQ_W8, M, N, K, sms);
+  plan.split = 1;
+  const char *why = nullptr;
+  return from_cuda(mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why),
+                   "stall gemm launch", why);
+}
+
+}  // extern "C"

@@ -1,0 +1,71 @@
+// Internal host-side interfaces between the C ABI layer (abi.cu) and the
+// kernel launchers.  Launchers assume validated arguments and return the
+// cudaError_t of their launch.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace mixq {
+
+constexpr int kGroup = 128;     // 4-bit group size along K
+constexpr int kBlockK = 128;    // K per pipeline stage (bytes of INT8)
+constexpr int kOutBlockK = 64;  // fp16 K per outlier stage (128 bytes)
+constexpr int kTileM = 128;     // output tile rows (tcgen05 M)
+
+inline int k_out_pad(int k_out) { return (k_out + 63) / 64 * 64; }
+
+// ---------------------------------------------------------------- quantize
+cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx,
+                                int K_out, float threshold, int8_t *Xq, float *s_x, void *X_out,
+                                uint32_t *bitmap, int32_t *flags, int32_t *status,
+                                cudaStream_t stream, int num_sms);
+
+// ----------------------------------------------------------------- prepack
+cudaError_t launch_prepack(int mode, const void *W, int N, int K, const int32_t *idx, int K_out,
+                           void *Wq, float *s_w, void *grp, void *W_out, int32_t *status,
+                           cudaStream_t stream);
+cudaError_t launch_unpack_w4(int N, int K, const void *Wq4, const void *grp, uint8_t *q,
+                             uint8_t *s2, uint8_t *z2, cudaStream_t stream);
+
+// -------------------------------------------------------------------- gemm
+struct GemmPlan {
+  int bn;     // output tile width (128 or 256)
+  int split;  // K split = cluster size along z (1..8)
+  int ctas;   // total CTAs launched
+};
+
+GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms);
+
+enum class Epi { kMixed = 0, kRawI32 = 1 };
+
+struct GemmArgs {
+  int mode;  // 0 = W8, 1 = W4G128
+  int M, N, K, K_out;
+  const int8_t *Xq;
+  const float *s_x;
+  const void *X_out;
+  const void *Wq;
+  const void *grp;
+  const float *s_w;
+  const void *W_out;
+  const int32_t *flags;
+  void *Y;  // fp16 [M][ldy] or int32 [M][ldy] (raw mode)
+  int ldy;
+  Epi epi;
+  int32_t *status;
+  uint64_t wait_limit_ns;
+  int debug_stall;  // producer issues nothing (timeout test)
+};
+
+cudaError_t launch_gemm(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
+                        const char **why);
+
+// Device properties cached per device.
+int device_sm_count(int dev);
+int device_cc_major(int dev);
+size_t device_max_smem_optin(int dev);
+
+}  // namespace mixq

@@ -1,0 +1,210 @@
+// Offline weight prepack for the MixQ layer.
+//
+// 8-bit (MixQ article "一键部署LLM混合精度推理…", 研究背景 Fig. 5): per output
+// channel symmetric INT8, a = max |W[n,:]| over all K, code = clamp(rint(w *
+// 127/a), -127, 127), s_w = a/127; outlier weight columns W[:, idx] gathered
+// in idx order (Fig. 11).
+//
+// 4-bit (QServe W4A8KV4 reading notes, 渐进量化 + group-wise; MixLLM page,
+// "MixLLM: Ein neuer Ansatz"): the INT8 codes are quantized again per group of
+// 128 along K with an integer scale s2 and zero z2 chosen so that the
+// effective weight (q - z2) * s2 always fits int8; the GEMM mainloop rebuilds
+// it with one integer multiply-add per four codes.  Packed layout: byte
+// (n, 64g + b) holds q[n, 128g + 8(b>>2) + (b&3)] in its low nibble and the
+// code four positions later in its high nibble, so a 32-bit word splits into
+// two words of four consecutive codes with one mask and one shift.
+#include <cuda_fp16.h>
+
+#include "internal.h"
+#include "ptx.cuh"
+
+namespace mixq {
+namespace {
+
+constexpr int kPThreads = 256;
+constexpr int kPWarps = kPThreads / 32;
+
+__device__ __forceinline__ float warp_max_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ int warp_min_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = min(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ int warp_max_i(int v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = max(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+template <bool kW4>
+__global__ void __launch_bounds__(kPThreads) prepack_kernel(
+    const __half *__restrict__ W, int N, int K, const int32_t *__restrict__ idx, int K_out,
+    int K_out_pad, void *__restrict__ Wq, float *__restrict__ s_w, __half2 *__restrict__ grp,
+    __half *__restrict__ W_out, int32_t *__restrict__ status) {
+  extern __shared__ int8_t psm[];  // kW4: the row's INT8 codes, then its 4-bit codes
+  __shared__ float s_red[kPWarps];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int nvec = K >> 3;
+  for (int n = blockIdx.x; n < N; n += gridDim.x) {
+    const uint4 *wr = reinterpret_cast<const uint4 *>(W + static_cast<size_t>(n) * K);
+    float a = 0.f;
+    for (int v = tid; v < nvec; v += kPThreads) {
+      const uint4 raw = __ldg(wr + v);
+      const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        a = fmaxf(a, fmaxf(fabsf(f.x), fabsf(f.y)));
+      }
+    }
+    a = warp_max_f(a);
+    if (lane == 0) s_red[warp] = a;
+    __syncthreads();
+    a = s_red[0];
+#pragma unroll
+    for (int w = 1; w < kPWarps; ++w) a = fmaxf(a, s_red[w]);
+    __syncthreads();
+    const float inv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
+    if (tid == 0) s_w[n] = __fdiv_rn(a, 127.f);
+
+    for (int v = tid; v < nvec; v += kPThreads) {
+      const uint4 raw = __ldg(wr + v);
+      const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
+      uint32_t word[2] = {0u, 0u};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 f = __half22float2(h[e]);
+        int q0 = max(-127, min(127, __float2int_rn(__fmul_rn(f.x, inv))));
+        int q1 = max(-127, min(127, __float2int_rn(__fmul_rn(f.y, inv))));
+        const uint32_t pair = (static_cast<uint32_t>(q0) & 0xFFu) |
+                              ((static_cast<uint32_t>(q1) & 0xFFu) << 8);
+        word[e >> 1] |= pair << (16 * (e & 1));
+      }
+      if (kW4) {
+        reinterpret_cast<uint2 *>(psm)[v] = make_uint2(word[0], word[1]);
+      } else {
+        reinterpret_cast<uint2 *>(static_cast<int8_t *>(Wq) + static_cast<size_t>(n) * K)[v] =
+            make_uint2(word[0], word[1]);
+      }
+    }
+    if (K_out_pad > 0) {
+      const __half *wh = W + static_cast<size_t>(n) * K;
+      for (int j = tid; j < K_out_pad; j += kPThreads) {
+        __half v = __ushort_as_half(0);
+        if (j < K_out) {
+          const int c = idx[j];
+          const bool ok = c >= 0 && c < K && (j == 0 || idx[j - 1] < c);
+          if (ok) v = wh[c];
+          else record_error(status, kErrInvalidArg);
+        }
+        W_out[static_cast<size_t>(n) * K_out_pad + j] = v;
+      }
+    }
+    if (kW4) {
+      __syncthreads();
+      // Level 2: one warp per group of 128 codes, four codes per lane.
+      const int groups = K / kGroup;
+      for (int g = warp; g < groups; g += kPWarps) {
+        int8_t *c = psm + g * kGroup + lane * 4;
+        int v[4], lo = 127, hi = -127;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[i] = c[i];
+          lo = min(lo, v[i]);
+          hi = max(hi, v[i]);
+        }
+        lo = warp_min_i(lo);
+        hi = warp_max_i(hi);
+        const int s2 = max(1, (hi - lo + 14) / 15);
+        const int z2 = max(0, min(15, __float2int_rn(__fdiv_rn(-static_cast<float>(lo),
+                                                                static_cast<float>(s2)))));
+        const int qlo = max(0, z2 - 128 / s2);
+        const int qhi = min(15, z2 + 127 / s2);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int r = __float2int_rn(__fdiv_rn(static_cast<float>(v[i]), static_cast<float>(s2)));
+          c[i] = static_cast<int8_t>(max(qlo, min(qhi, r + z2)));
+        }
+        if (lane == 0)
+          grp[static_cast<size_t>(g) * N + n] =
+              __halves2half2(__int2half_rn(s2), __int2half_rn(z2));
+      }
+      __syncthreads();
+      // Pack: 4 output bytes (one 32-bit word = 8 codes) per thread and step.
+      uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(Wq) +
+                                                   static_cast<size_t>(n) * (K / 2));
+      for (int wi = tid; wi < K / 8; wi += kPThreads) {
+        const int8_t *src = psm + wi * 8;  // codes k = 8wi .. 8wi+7
+        uint32_t word = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint32_t byte = (static_cast<uint32_t>(src[i]) & 0xFu) |
+                                ((static_cast<uint32_t>(src[i + 4]) & 0xFu) << 4);
+          word |= byte << (8 * i);
+        }
+        dst[wi] = word;
+      }
+      __syncthreads();
+    }
+  }
+}
+
+__global__ void unpack_w4_kernel(int N, int K, const uint8_t *__restrict__ Wq4,
+                                 const __half2 *__restrict__ grp, uint8_t *__restrict__ q,
+                                 uint8_t *__restrict__ s2, uint8_t *__restrict__ z2) {
+  const size_t total = static_cast<size_t>(N) * K;
+  const int groups = K / kGroup;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int n = static_cast<int>(i / K), k = static_cast<int>(i % K);
+    const int g = k / kGroup, r = k % kGroup;
+    const int b = 4 * (r >> 3) + (r & 3);
+    const uint8_t byte = Wq4[static_cast<size_t>(n) * (K / 2) + g * 64 + b];
+    q[i] = (r & 4) ? (byte >> 4) : (byte & 0xF);
+    if (r == 0) {
+      const float2 sz = __half22float2(grp[static_cast<size_t>(g) * N + n]);
+      s2[static_cast<size_t>(n) * groups + g] = static_cast<uint8_t>(sz.x);
+      z2[static_cast<size_t>(n) * groups + g] = static_cast<uint8_t>(sz.y);
+    }
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_prepack(int mode, const void *W, int N, int K, const int32_t *idx, int K_out,
+                           void *Wq, float *s_w, void *grp, void *W_out, int32_t *status,
+                           cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  const int grid = N < 4096 ? N : 4096;
+  if (mode == 0) {
+    prepack_kernel<false><<<grid, kPThreads, 0, stream>>>(
+        static_cast<const __half *>(W), N, K, idx, K_out, k_out_pad(K_out), Wq, s_w, nullptr,
+        static_cast<__half *>(W_out), status);
+  } else {
+    const size_t smem = static_cast<size_t>(K);
+    cudaError_t e = cudaFuncSetAttribute(prepack_kernel<true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem < 48 * 1024 ? 48 * 1024 : smem));
+    if (e != cudaSuccess) return e;
+    prepack_kernel<true><<<grid, kPThreads, smem, stream>>>(
+        static_cast<const __half *>(W), N, K, idx, K_out, k_out_pad(K_out), Wq, s_w,
+        static_cast<__half2 *>(grp), static_cast<__half *>(W_out), status);
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_unpack_w4(int N, int K, const void *Wq4, const void *grp, uint8_t *q,
+                             uint8_t *s2, uint8_t *z2, cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  unpack_w4_kernel<<<1024, 256, 0, stream>>>(N, K, static_cast<const uint8_t *>(Wq4),
+                                             static_cast<const __half2 *>(grp), q, s2, z2);
+  return cudaGetLastError();
+}
+
+}  // namespace mixq

@@ -1,0 +1,99 @@
+"""The C ABI library on a machine without a GPU: it loads, exports every symbol
+include/mixq.h declares, and does its host-side work (argument checks, size
+queries, launch planning) without touching a device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import mixed_precision_quantized_mixq_b200 as mq
+from mixed_precision_quantized_mixq_b200 import build as mqbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    mqbuild.build()
+    return mq.lib()
+
+
+def _declared():
+    with open(os.path.join(ROOT, "include", "mixq.h")) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"\b(mixq_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol(lib):
+    names = _declared()
+    assert len(names) >= 11
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(mq._SIGNATURES), "binding signatures out of sync with the header"
+
+
+def test_version(lib):
+    assert lib.mixq_version() == 100
+
+
+def test_prepack_size(lib):
+    assert mq.mixq_prepack_size(mq.MIXQ_W8, 256, 512, 4) == (256 * 512, 0, 2 * 256 * 64)
+    assert mq.mixq_prepack_size(mq.MIXQ_W4G128, 256, 512, 65) == (256 * 256, 4 * 256 * 4,
+                                                                  2 * 256 * 128)
+    assert mq.mixq_prepack_size(mq.MIXQ_W8, 128, 128, 0)[2] == 0
+
+
+@pytest.mark.parametrize("N,K,K_out", [(100, 128, 0), (128, 100, 0), (0, 128, 0), (128, 128, 129),
+                                       (128, 128, -1)])
+def test_shape_rules(lib, N, K, K_out):
+    with pytest.raises(mq.MixqError) as e:
+        mq.mixq_prepack_size(mq.MIXQ_W8, N, K, K_out)
+    assert e.value.status == 2
+    assert "must" in lib.mixq_last_error().decode()
+
+
+def test_bad_mode(lib):
+    with pytest.raises(mq.MixqError) as e:
+        mq.mixq_prepack_size(7, 128, 128, 0)
+    assert e.value.status == 1
+
+
+def test_host_checks_come_before_device_checks(lib):
+    # misaligned pointers are reported without any device access
+    rc = lib.mixq_gemm_w8a8o16(4, 256, 256, 0, 0x1001, 0x2000, None, 0x3000, 0x4000, None, None,
+                               0x5000, 256, None, None)
+    assert rc == 3
+    rc = lib.mixq_gemm_w8a8o16(4, 256, 256, 0, None, 0x2000, None, 0x3000, 0x4000, None, None,
+                               0x5000, 256, None, None)
+    assert rc == 1
+    rc = lib.mixq_gemm_w8a8o16(4, 256, 256, 0, 0x1000, 0x2000, None, 0x3000, 0x4000, None, None,
+                               0x5000, 250, None, None)
+    assert rc == 1
+    rc = lib.mixq_quantize_act(0x1000, 4, 256, 256, None, 0, ctypes.c_float(-1.0), 0x2000, 0x3000,
+                               None, 0x4000, 0x5000, None, None)
+    assert rc == 1
+
+
+def test_no_device_reported(lib):
+    import torch
+    if torch.cuda.is_available():
+        pytest.skip("a GPU is present")
+    rc = lib.mixq_gemm_w8a8o16(4, 256, 256, 0, 0x1000, 0x2000, None, 0x3000, 0x4000, None, None,
+                               0x5000, 256, None, None)
+    assert rc == 6
+    assert "device" in lib.mixq_last_error().decode()
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 11008, 4096), (64, 4096, 11008),
+                                   (512, 4096, 4096), (2048, 11008, 4096), (8192, 11008, 4096),
+                                   (512, 28672, 8192), (512, 8192, 28672)])
+def test_gemm_plan(lib, M, N, K):
+    bn, split, ctas = mq.mixq_gemm_plan(mq.MIXQ_W8, M, N, K, 148)
+    assert bn in (128, 256) and 1 <= split <= 8 and split <= K // 128
+    assert ctas == -(-M // 128) * -(-N // bn) * split
+    if M <= 64:
+        # decode: K is split across a cluster so most SMs stream weights
+        assert ctas >= 100
+    if M >= 2048:
+        assert split == 1
