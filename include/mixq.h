@@ -28,6 +28,11 @@
  *   - mixq_last_error() returns a thread-local description of the last
  *     non-OK status returned on the calling thread.
  *   - Calls that share output buffers must not overlap on the GPU.
+ *   - Kernels are launched with programmatic dependent launch: a call's
+ *     kernels may begin while the preceding kernel on the stream finishes, and
+ *     wait for it before reading its outputs.  The gemm calls start streaming
+ *     the prepacked weights (Wq, grp) before that wait, so those buffers must
+ *     not be written by the kernel immediately preceding the gemm call.
  *
  * Shape rules (MIXQ_ERR_UNSUPPORTED_SHAPE otherwise): K % 128 == 0, K > 0,
  * N % 128 == 0, N > 0, M >= 0, 0 <= K_out <= K.  K_out_pad is K_out rounded up
@@ -65,8 +70,8 @@ int mixq_version(void);
 
 /*
  * Sizes of the prepacked weight buffers for mode, N, K, K_out (host only).
- *   *wq_bytes   MIXQ_W8: N*K (int8 codes, row-major [N][K]).
- *               MIXQ_W4G128: N*K/2 (two 4-bit codes per byte, see below).
+ *   *wq_bytes   MIXQ_W8: N*K (int8 codes, tiled, see mixq_prepack_weights).
+ *               MIXQ_W4G128: N*K/2 (two 4-bit codes per byte, tiled).
  *   *grp_bytes  MIXQ_W4G128: 4*N*(K/128) (one fp16 pair (s2, z2) per group,
  *               group-major [K/128][N]); MIXQ_W8: 0.
  *   *wout_bytes 2*N*K_out_pad (fp16 [N][K_out_pad]).
@@ -81,10 +86,18 @@ mixq_status mixq_prepack_size(int mode, int N, int K, int K_out, size_t *wq_byte
  *   W      fp16 [N][K]           input weights (read only)
  *   idx    int32 [K_out]          outlier channels, sorted ascending, unique,
  *                                 inside [0, K) (checked on the device)
- *   Wq     MIXQ_W8: int8 [N][K], code = clamp(rint(W * 127/a), -127, 127) with
- *          a = max_k |W[n,k]| over all K; MIXQ_W4G128: packed level-2 codes,
- *          byte (n, g*64 + b) holds q[n, 128g + 8(b>>2) + (b&3)] in its low
- *          nibble and q[n, same + 4] in its high nibble.
+ *   Wq     codes in a tiled layout made for the GEMM's bulk copies (QServe
+ *          notes, compute-aware weight reordering): tiles of 128 output
+ *          channels x 128 K, tile (n/128, k/128) at tile index
+ *          (n/128)*(K/128) + k/128, each tile contiguous.
+ *          MIXQ_W8: code = clamp(rint(W * 127/a), -127, 127) with a =
+ *          max_k |W[n,k]| over all K; 16 KB tiles, row r = n%128 at r*128, the
+ *          16-byte chunk of K offsets 16j..16j+15 at chunk position j^(r%8).
+ *          MIXQ_W4G128: 4-bit level-2 codes q; 8 KB tiles, row r at r*64, the
+ *          16-byte chunk c (K offsets 32c..32c+31) at chunk position
+ *          c^((r/2)%4); inside it byte 4w+i holds q at K offset 32c+8w+i in
+ *          its low nibble and q at 32c+8w+4+i in its high nibble.
+ *          mixq_debug_unpack_w8 / _w4 return the logical codes.
  *   s_w    fp32 [N]               a / 127
  *   grp    MIXQ_W4G128 only (else NULL): fp16 pairs (s2, z2) at [g][n], with
  *          s2 = max(1, ceil((hi-lo)/15)), z2 = clamp(rint(-lo/s2), 0, 15) over
@@ -118,7 +131,10 @@ mixq_status mixq_prepack_weights(int mode, const void *W, int N, int K, const in
  *                  by the call and read 0 when it completes.  gemm calls read
  *                  flags[0] on the device to skip the FP16 slice when no
  *                  token is mixed.
- * Launches two kernels (a 1-block reset of bitmap/flags, then the main pass).
+ * K must not exceed 32768 (a token's row is held in registers).
+ * For M <= 32 G tokens (G = 2 when K <= 8192, else 1) one thread-block
+ * cluster covers the matrix and the call is one kernel; for larger M it is a
+ * 1-block reset of bitmap/flags followed by the main pass.
  */
 mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx, int K_out,
                               float threshold, int8_t *Xq, float *s_x, void *X_out,
@@ -157,9 +173,11 @@ mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
 
 /*
  * The launch plan the gemm calls use for a shape (host only, no GPU needed):
- * output tile width *bn (128 or 256 columns; tiles are 128 rows high), the
- * K-split factor *split (thread-block cluster size along K, 1..8) and the
- * number of CTAs *ctas.  num_sms <= 0 means "query the current device".
+ * output tile width *bn (32, 64, 128 or 256 columns; tiles are 128 rows
+ * high), the K-split factor *split (thread-block cluster size along K, 1..8)
+ * and the number of CTAs *ctas.  num_sms <= 0 means "query the current
+ * device" (and its cluster occupancy).  For M <= 64 and bn <= 128 the plan
+ * runs the small-M variant (token-sized A slots, two CTAs per SM).
  */
 mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, int *split,
                            int *ctas);
@@ -167,11 +185,22 @@ mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, 
 /*
  * Test-only: the gemm mainloop alone, raw INT32 accumulators out
  * (acc int32 [M][ldacc]).  mode MIXQ_W8 uses Wq; MIXQ_W4G128 uses Wq4 + grp.
- * bn/split override the plan when > 0.
+ * bn/split override the plan when > 0 (bn 32 and 64 need M <= 64; with
+ * M <= 64 and bn <= 128 the small-M variant runs).
  */
 mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq, const void *Wq,
                                 const void *grp, int32_t *acc, int ldacc, int bn, int split,
                                 int32_t *status, void *stream);
+
+/* Test-only: how many thread-block clusters of the gemm kernel (mode, tile
+ * width bn, K-split cluster size split, small_m = the M <= 64 variant that
+ * fits two CTAs per SM, bn 32/64/128; bn 32/64 exist only as small_m) the
+ * current device runs at once. */
+mixq_status mixq_debug_max_active_clusters(int mode, int bn, int split, int small_m,
+                                           int *clusters);
+
+/* Test-only: logical INT8 codes back from the tiled W8 layout: out int8 [N][K]. */
+mixq_status mixq_debug_unpack_w8(int N, int K, const void *Wq, int8_t *out, void *stream);
 
 /* Test-only: logical 4-bit codes back from the packed layout:
  * q uint8 [N][K], s2/z2 uint8 [N][K/128]. */

@@ -38,6 +38,8 @@ _SIGNATURES = {
                                _VP, _VP]),
     "mixq_gemm_plan": (_I, [_I, _I, _I, _I, _I, _c.POINTER(_I), _c.POINTER(_I), _c.POINTER(_I)]),
     "mixq_debug_gemm_i32": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _I, _I, _I, _VP, _VP]),
+    "mixq_debug_max_active_clusters": (_I, [_I, _I, _I, _I, _c.POINTER(_I)]),
+    "mixq_debug_unpack_w8": (_I, [_I, _I, _VP, _VP, _VP]),
     "mixq_debug_unpack_w4": (_I, [_I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "mixq_debug_gemm_stall": (_I, [_I, _I, _I, _VP, _VP, _VP, _VP, _VP, _I, _U64, _VP, _VP]),
 }
@@ -137,6 +139,16 @@ def mixq_debug_gemm_i32(mode, Xq, Wq, grp, acc, N, bn=0, split=0, status=None, s
                                      acc.stride(0), bn, split, _ptr(status), _stream(stream)))
 
 
+def mixq_debug_max_active_clusters(mode: int, bn: int, split: int, small_m: int = 0) -> int:
+    n = _I()
+    _check(lib().mixq_debug_max_active_clusters(mode, bn, split, small_m, ctypes.byref(n)))
+    return n.value
+
+
+def mixq_debug_unpack_w8(N, K, Wq, out, stream=None):
+    _check(lib().mixq_debug_unpack_w8(N, K, _ptr(Wq), _ptr(out), _stream(stream)))
+
+
 def mixq_debug_unpack_w4(N, K, Wq4, grp, q, s2, z2, status=None, stream=None):
     _check(lib().mixq_debug_unpack_w4(N, K, _ptr(Wq4), _ptr(grp), _ptr(q), _ptr(s2), _ptr(z2),
                                       _ptr(status), _stream(stream)))
@@ -165,7 +177,7 @@ class PackedWeights:
     N: int
     K: int
     idx: "object"      # int32 [K_out]
-    Wq: "object"       # int8 [N, K] (W8) or uint8 [N, K/2] (W4)
+    Wq: "object"       # tiled codes: int8 [N*K] (W8) or uint8 [N*K/2] (W4), see mixq.h
     s_w: "object"      # fp32 [N]
     grp: "object"      # fp16 [K/128, N, 2] (W4) or None
     W_out: "object"    # fp16 [N, K_out_pad] or None
@@ -195,10 +207,10 @@ def prepack(W, idx, mode: int = MIXQ_W8, status=None, stream=None) -> PackedWeig
     idx = torch.as_tensor(idx, dtype=torch.int32, device=dev).contiguous()
     ko = idx.numel()
     if mode == MIXQ_W8:
-        Wq = torch.empty((N, K), dtype=torch.int8, device=dev)
+        Wq = torch.empty(N * K, dtype=torch.int8, device=dev)
         grp = None
     else:
-        Wq = torch.empty((N, K // 2), dtype=torch.uint8, device=dev)
+        Wq = torch.empty(N * K // 2, dtype=torch.uint8, device=dev)
         grp = torch.empty((K // GROUP, N, 2), dtype=torch.float16, device=dev)
     s_w = torch.empty(N, dtype=torch.float32, device=dev)
     W_out = torch.empty((N, k_out_pad(ko)), dtype=torch.float16, device=dev) if ko else None

@@ -144,6 +144,9 @@ mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_
                               void *stream) {
   mixq_status s = check_shape(M, 128, K, K_out);
   if (s != MIXQ_OK) return s;
+  if (K > mixq::quantize_max_k())
+    return fail(MIXQ_ERR_UNSUPPORTED_SHAPE, "K = %d exceeds %d for mixq_quantize_act", K,
+                mixq::quantize_max_k());
   if (ldx < K || ldx % 8) return fail(MIXQ_ERR_INVALID_ARG, "ldx = %d must be >= K and a multiple of 8", ldx);
   if (!(threshold >= 0.f) || threshold != threshold)
     return fail(MIXQ_ERR_INVALID_ARG, "threshold must be a finite value >= 0");
@@ -202,10 +205,11 @@ static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const i
   a.epi = mixq::Epi::kMixed;
   a.status = status;
   a.wait_limit_ns = kDefaultWaitNs;
-  const mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms);
+  const mixq::GemmPlan plan =
+      mixq::plan_gemm(mode, M, N, K, sms, mixq::device_cluster_limits(mode));
   const char *why = nullptr;
-  return from_cuda(mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why),
-                   "gemm launch", why);
+  const cudaError_t e = mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why);
+  return from_cuda(e, "gemm launch", why);
 }
 
 mixq_status mixq_gemm_w8a8o16(int M, int N, int K, int K_out, const int8_t *Xq, const float *s_x,
@@ -229,14 +233,29 @@ mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, 
   if (mode != MIXQ_W8 && mode != MIXQ_W4G128) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
   mixq_status s = check_shape(M, N, K, 0);
   if (s != MIXQ_OK) return s;
+  const mixq::ClusterLimits *limits = nullptr;
   if (num_sms <= 0) {
     s = check_device(&num_sms);
     if (s != MIXQ_OK) return s;
+    limits = mixq::device_cluster_limits(mode);
   }
-  const mixq::GemmPlan p = mixq::plan_gemm(mode, M, N, K, num_sms);
+  const mixq::GemmPlan p = mixq::plan_gemm(mode, M, N, K, num_sms, limits);
   if (bn) *bn = p.bn;
   if (split) *split = p.split;
   if (ctas) *ctas = p.ctas;
+  return ok();
+}
+
+mixq_status mixq_debug_max_active_clusters(int mode, int bn, int split, int small_m,
+                                           int *clusters) {
+  if ((mode != MIXQ_W8 && mode != MIXQ_W4G128) ||
+      (bn != 32 && bn != 64 && bn != 128 && bn != 256) || split < 1 || split > 8 || !clusters ||
+      (small_m && bn == 256) || (!small_m && bn < 128))
+    return fail(MIXQ_ERR_INVALID_ARG, "bad mode/bn/split/small_m/pointer");
+  mixq_status s = check_device(nullptr);
+  if (s != MIXQ_OK) return s;
+  *clusters = mixq::gemm_max_active_clusters(mode, bn, split, small_m);
+  if (*clusters < 0) return fail(MIXQ_ERR_CUDA, "cudaOccupancyMaxActiveClusters failed");
   return ok();
 }
 
@@ -247,7 +266,10 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   mixq_status s = check_shape(M, N, K, 0);
   if (s != MIXQ_OK) return s;
   if (ldacc < N || ldacc % 4) return fail(MIXQ_ERR_INVALID_ARG, "ldacc = %d must be >= N and a multiple of 4", ldacc);
-  if (bn != 0 && bn != 128 && bn != 256) return fail(MIXQ_ERR_INVALID_ARG, "bn = %d", bn);
+  if (bn != 0 && bn != 32 && bn != 64 && bn != 128 && bn != 256)
+    return fail(MIXQ_ERR_INVALID_ARG, "bn = %d", bn);
+  if ((bn == 32 || bn == 64) && M > 64)
+    return fail(MIXQ_ERR_INVALID_ARG, "bn = %d needs M <= 64", bn);
   if (split < 0 || split > 8)
     return fail(MIXQ_ERR_INVALID_ARG, "split = %d", split);
   if (split > K / 128) return fail(MIXQ_ERR_UNSUPPORTED_SHAPE, "split %d exceeds K/128", split);
@@ -259,9 +281,10 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   int sms = 0;
   s = check_device(&sms);
   if (s != MIXQ_OK) return s;
-  mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms);
+  mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms, mixq::device_cluster_limits(mode));
   if (bn) plan.bn = bn;
   if (split) plan.split = split;
+  if (bn || split) plan.small_m = (M <= 64 && plan.bn <= 128) ? 1 : 0;
   mixq::GemmArgs a{};
   a.mode = mode;
   a.M = M;
@@ -276,8 +299,18 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   a.status = status;
   a.wait_limit_ns = kDefaultWaitNs;
   const char *why = nullptr;
-  return from_cuda(mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why),
-                   "debug gemm launch", why);
+  const cudaError_t e = mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why);
+  return from_cuda(e, "debug gemm launch", why);
+}
+
+mixq_status mixq_debug_unpack_w8(int N, int K, const void *Wq, int8_t *out, void *stream) {
+  mixq_status s = check_shape(0, N, K, 0);
+  if (s != MIXQ_OK) return s;
+  if (!Wq || !out) return fail(MIXQ_ERR_INVALID_ARG, "null pointer");
+  s = check_device(nullptr);
+  if (s != MIXQ_OK) return s;
+  return from_cuda(mixq::launch_unpack_w8(N, K, Wq, out, static_cast<cudaStream_t>(stream)),
+                   "unpack launch");
 }
 
 mixq_status mixq_debug_unpack_w4(int N, int K, const void *Wq4, const void *grp, uint8_t *q,
@@ -321,11 +354,13 @@ mixq_status mixq_debug_gemm_stall(int M, int N, int K, const int8_t *Xq, const v
   a.status = status;
   a.wait_limit_ns = wait_limit_ns;
   a.debug_stall = 1;
-  mixq::GemmPlan plan = mixq::plan_gemm(MIXQ_W8, M, N, K, sms);
+  mixq::GemmPlan plan = mixq::plan_gemm(MIXQ_W8, M, N, K, sms, nullptr);
   plan.split = 1;
+  plan.bn = 128;
+  plan.small_m = M <= 64 ? 1 : 0;
   const char *why = nullptr;
-  return from_cuda(mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why),
-                   "stall gemm launch", why);
+  const cudaError_t e = mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why);
+  return from_cuda(e, "stall gemm launch", why);
 }
 
 }  // extern "C"

@@ -39,27 +39,59 @@
 namespace mixq {
 namespace {
 
-template <int BN, bool W4>
+// Shared-memory plan (all offsets multiples of 1 KB):
+//   ring  = [A slots: stages x a_stride][B stages: stages x kBStage]
+//   then    barriers (1 KB), s_w of the tile (1 KB), s_x of the tile (512 B).
+// An A slot holds the Xq (or X_out) tile of one stage: a_stride = 16 KB (128
+// rows) normally.  With SM ("small M", at most 64 tokens) a slot holds only
+// the token rows (M rounded up to 8, 128 bytes each); the MMA still reads 128
+// rows, and rows past the slot run into the next slots or the B stages --
+// rows of D that are never stored.  That keeps a decode-sized CTA near
+// 100 KB, so one CTA of the next kernel fits beside it on the SM (two CTAs'
+// TMEM, 2 x 2 x 128 columns, fit too) and, launched early by programmatic
+// dependent launch, streams its weights while this kernel finishes.
+// A B stage holds the INT8 weight tile (or the W_out tile), and for W4 the
+// packed 4-bit codes and their group constants.
+template <int BN, bool W4, bool SM>
 struct Cfg {
-  static constexpr int kA = kTileM * kBlockK;             // A stage: 128 rows x 128 B
-  static constexpr int kB = BN * kBlockK;                 // B stage: BN rows x 128 B
-  static constexpr int kP = W4 ? BN * (kBlockK / 2) : 0;  // packed 4-bit codes
+  static constexpr int kMaxStages = 8;
+  static constexpr int kB = BN * kBlockK;                  // INT8 / fp16 B tile
+  static constexpr int kP = W4 ? BN * (kBlockK / 2) : 0;   // packed 4-bit codes
   static constexpr int kG = W4 ? ((BN * 4 + 1023) / 1024) * 1024 : 0;  // (s2,z2) per row
-  static constexpr int kStage = kA + kB + kP + kG;
+  static constexpr int kBStage = kB + kP + kG;
+  // full-size (not SM) stage count; SM stage counts are chosen at launch
   static constexpr int kStages = W4 ? (BN == 256 ? 3 : 5) : (BN == 256 ? 4 : 6);
-  static constexpr int kThreads = W4 ? 256 : 128;
+  static constexpr int kExpandThreads = W4 ? (SM ? 128 : 256) : 0;  // warps 4..
+  static constexpr int kThreads = 128 + kExpandThreads;
+  static constexpr int kMinBlocks = SM ? 2 : 1;
   static constexpr int kTmemCols = 2 * BN;  // INT32 acc [0,BN), FP32 outlier acc [BN,2BN)
-  static constexpr int kBarBytes = 1024;
-  static constexpr int kSmem = kStages * kStage + kBarBytes + 1024;  // + alignment slack
-  // cluster reduction buffers (reuse the stage ring after the mainloop)
-  static constexpr int kCW = 128;
+  static constexpr int kExtra = 1024 + 1024 + 512;  // barriers, s_w, s_x
+  // weight bytes of one 128-row tile of one K block, and of one weight row
+  static constexpr int kSubW = W4 ? 128 * (kBlockK / 2) : 128 * kBlockK;
+  static constexpr int kRowW = W4 ? kBlockK / 2 : kBlockK;
+  static constexpr int kSubRows = BN < 128 ? BN : 128;  // rows per bulk copy
+  static_assert(BN == 32 || BN == 64 || BN == 128 || BN == 256, "tile width");
+  static_assert(BN >= 128 || SM, "narrow tiles are small-M only");
+  // cluster reduction buffers (reuse the ring after the mainloop)
+  static constexpr int kCW = BN < 128 ? BN : 128;  // columns per reduction round
   static constexpr int kPitch = kCW + 4;  // words; +4 keeps 16-byte rows off one bank group
-  static_assert(2 * kTileM * kPitch * 4 <= kStages * kStage, "reduction buffers do not fit");
-  static_assert(kSmem <= 232448, "shared memory budget");
+  static constexpr int kRedRows = SM ? 64 : 128;
+  static constexpr int kRedBytes = 2 * kRedRows * kPitch * 4;
+  __host__ __device__ static constexpr int ring_bytes(int stages, int a_stride) {
+    return stages * (a_stride + kBStage);
+  }
+  __host__ __device__ static constexpr int smem_bytes(int stages, int a_stride) {
+    return ring_bytes(stages, a_stride) + kExtra + 1024;  // + alignment slack
+  }
 };
 
 struct KParams {
   int M, N, K, K_out_pad;
+  int a_rows;            // rows of the A / X_out TMA box (M rounded up to 8, at most 128)
+  int a_stride;          // bytes of one A slot
+  int stages;            // pipeline depth
+  const uint8_t *wq;     // tiled weight codes (W8: 16 KB tiles, W4: 8 KB tiles)
+  const uint8_t *grp;    // W4 group constants [K/128][N] (s2, z2) fp16 pairs
   const float *s_x;
   const float *s_w;
   const int32_t *flags;
@@ -84,26 +116,38 @@ __device__ __forceinline__ uint32_t expand4(uint32_t nibbles, uint32_t s2, uint3
   return (nibbles * s2 + c) ^ 0x80808080u;
 }
 
-template <int BN, bool W4, bool RAW>
-__global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
+// Whether the FP16 outlier slice runs: some token is mixed (flags[0] > 0), or
+// the caller passed no flags.  Read after griddep_wait().
+__device__ __forceinline__ int outliers_present(const KParams &p, bool raw) {
+  if (raw || p.K_out_pad == 0) return 0;
+  return p.flags ? (*reinterpret_cast<const volatile int32_t *>(p.flags) > 0) : 1;
+}
+
+template <int BN, bool W4, bool SM, bool RAW>
+__global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kMinBlocks)
     mixq_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,   // Xq   [M][K] int8
-                     const __grid_constant__ CUtensorMap tm_b,   // Wq [N][K] int8 | Wq4 [N][K/2]
-                     const __grid_constant__ CUtensorMap tm_g,   // grp [K/128][N] (s2,z2)
                      const __grid_constant__ CUtensorMap tm_xo,  // X_out [M][K_out_pad] fp16
                      const __grid_constant__ CUtensorMap tm_wo,  // W_out [N][K_out_pad] fp16
                      const KParams p) {
-  using C = Cfg<BN, W4>;
+  using C = Cfg<BN, W4, SM>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const int stages = p.stages;
   uint8_t *ring = smem;
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kStages * C::kStage);
+  uint8_t *b_region = ring + stages * p.a_stride;
+  auto a_slot = [&](int s) { return ring + s * p.a_stride; };
+  auto b_slot = [&](int s) { return b_region + s * C::kBStage; };
+  uint8_t *extra = ring + C::ring_bytes(stages, p.a_stride);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(extra);
   uint64_t *full = bars;
-  uint64_t *empty = bars + C::kStages;
-  uint64_t *ready = bars + 2 * C::kStages;
-  uint64_t *accum_full = bars + 3 * C::kStages;
+  uint64_t *empty = bars + C::kMaxStages;
+  uint64_t *ready = bars + 2 * C::kMaxStages;
+  uint64_t *accum_full = bars + 3 * C::kMaxStages;
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(accum_full + 1);
-  int *s_misc = reinterpret_cast<int *>(tmem_holder + 1);  // err, any_out, consumed, issued
+  int *s_misc = reinterpret_cast<int *>(tmem_holder + 1);  // err, -, consumed, issued
+  float *s_sw = reinterpret_cast<float *>(extra + 1024);   // [BN]
+  float *s_sx = reinterpret_cast<float *>(extra + 2048);   // [128]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kTileM;
@@ -113,25 +157,72 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
   const int KB = p.K / kBlockK;
   const int kb_begin = static_cast<int>(static_cast<long long>(rank) * KB / S);
   const int kb_end = static_cast<int>(static_cast<long long>(rank + 1) * KB / S);
+  const int n_i8 = kb_end - kb_begin;                   // INT8 jobs come first
+  // weight rows of the tile come in n_sub slices of kSubRows rows (a slice of
+  // one 128-row weight tile when BN < 128; for BN = 256 the second slice is
+  // absent in the last column tile when N % 256 == 128)
+  const int n_sub = BN < 128 ? 1 : min(BN, p.N - n0) / 128;
+  const uint32_t a_bytes = static_cast<uint32_t>(p.a_rows) * kBlockK;
+  const uint32_t b_bytes = static_cast<uint32_t>(n_sub) * C::kSubRows * (C::kRowW + (W4 ? 4 : 0));
+  const int pre = n_i8 < stages ? n_i8 : stages;        // stages whose weights go out early
+
+  // address of the weight slice h of K block kb, and of its group constants
+  auto w_src = [&](int kb, int h) {
+    const int nrow = n0 + h * 128;
+    const size_t tile = static_cast<size_t>(nrow / 128) * KB + kb;
+    return p.wq + tile * C::kSubW + (nrow % 128) * C::kRowW;
+  };
+  auto g_src = [&](int kb, int h) {
+    return p.grp + (static_cast<size_t>(kb) * p.N + n0 + h * 128) * 4;
+  };
+  // weights of INT8 job j (K block kb_begin + j) into stage s: one bulk copy
+  // per weight slice (plus its group constants for W4)
+  auto issue_b = [&](int j, int s, uint64_t pol_b) {
+    const int kb = kb_begin + j;
+    uint8_t *sB = b_slot(s);
+    uint8_t *dstW = W4 ? sB + C::kB : sB;
+    uint8_t *dstG = sB + C::kB + C::kP;
+    for (int h = 0; h < n_sub; ++h) {
+      bulk_load(dstW + h * 128 * C::kRowW, w_src(kb, h), C::kSubRows * C::kRowW, &full[s], pol_b);
+      if (W4) bulk_load(dstG + h * 128 * 4, g_src(kb, h), C::kSubRows * 4, &full[s], pol_b);
+    }
+  };
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::kStages; ++i) {
+    for (int i = 0; i < stages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
-      if (W4) mbar_init(&ready[i], 128);
+      if (W4) mbar_init(&ready[i], C::kExpandThreads);
     }
     mbar_init(accum_full, 1);
     fence_mbar_init();
-    int any_out = 0;
-    if (!RAW && p.K_out_pad > 0) any_out = p.flags ? (p.flags[0] > 0) : 1;
     s_misc[0] = 0;
-    s_misc[1] = any_out;
+    s_misc[1] = 0;
     s_misc[2] = 0;
     s_misc[3] = 0;
+    // The weights do not depend on the preceding kernel: start streaming them
+    // first, before the rest of the set-up and before waiting for that kernel.
+    if (!p.debug_stall) {
+      const uint64_t pol_b = p.b_streamed ? policy_evict_first() : policy_evict_last();
+      for (int j = 0; j < pre; ++j) {
+        mbar_arrive_expect_tx(&full[j], a_bytes + b_bytes);
+        issue_b(j, j, pol_b);
+      }
+      // When this CTA is the only reader of its weights (one row tile of
+      // tokens), pull the rest of its weight slice into L2 now as well: the
+      // HBM stream then runs ahead of the pipeline, across the wait for the
+      // preceding kernel and across this CTA's own stage recycling.
+      if (p.b_streamed) {
+        for (int j = pre; j < n_i8; ++j) {
+          for (int h = 0; h < n_sub; ++h) {
+            prefetch_l2(w_src(kb_begin + j, h), C::kSubRows * C::kRowW);
+            if (W4) prefetch_l2(g_src(kb_begin + j, h), C::kSubRows * 4);
+          }
+        }
+      }
+    }
     tma_prefetch_desc(&tm_a);
-    tma_prefetch_desc(&tm_b);
-    if (W4) tma_prefetch_desc(&tm_g);
-    if (any_out && rank == 0) {
+    if (!RAW && p.K_out_pad > 0 && rank == 0) {
       tma_prefetch_desc(&tm_xo);
       tma_prefetch_desc(&tm_wo);
     }
@@ -140,14 +231,15 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
     tmem_alloc(tmem_holder, C::kTmemCols);
     tmem_relinquish();
   }
+  if (!RAW && (warp == 2 || warp == 3)) {
+    // per-channel weight scales of the tile (read only here, never in the epilogue loop)
+    for (int i = threadIdx.x - 64; i < BN; i += 64) s_sw[i] = n0 + i < p.N ? p.s_w[n0 + i] : 0.f;
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (threadIdx.x == 0) griddep_launch_dependents();
   const uint32_t tmem_base = *tmem_holder;
-  const int any_out = s_misc[1];
-  const bool do_out = any_out && rank == 0;
-  const int n_out = do_out ? p.K_out_pad / kOutBlockK : 0;
-  const int njobs = n_out + (kb_end - kb_begin);
   int *s_err = &s_misc[0];
 
   if (warp == 0) {
@@ -155,34 +247,28 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
     if (lane == 0 && !p.debug_stall) {
       const uint64_t pol_a = policy_evict_last();
       const uint64_t pol_b = p.b_streamed ? policy_evict_first() : policy_evict_last();
-      int issued = 0;
-      for (int j = 0; j < njobs; ++j) {
-        const int s = j % C::kStages;
-        const uint32_t ph = (j / C::kStages) & 1;
+      griddep_wait();
+      const int n_out = (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
+      const int njobs = n_i8 + n_out;
+      for (int j = 0; j < pre; ++j)
+        tma_load_2d(a_slot(j), &tm_a, &full[j], (kb_begin + j) * kBlockK, m0, pol_a);
+      int issued = pre;
+      for (int j = pre; j < njobs; ++j) {
+        const int s = j % stages;
+        const uint32_t ph = (j / stages) & 1;
         if (!mbar_wait(&empty[s], ph ^ 1, p.wait_limit_ns)) {
           fail(s_err, p.status);
           break;
         }
-        uint8_t *sA = ring + s * C::kStage;
-        uint8_t *sB = sA + C::kA;
-        uint8_t *sP = sB + C::kB;
-        uint8_t *sG = sP + C::kP;
-        if (j < n_out) {
-          mbar_arrive_expect_tx(&full[s], C::kA + C::kB);
-          tma_load_2d(sA, &tm_xo, &full[s], j * kOutBlockK, m0, pol_a);
-          tma_load_2d(sB, &tm_wo, &full[s], j * kOutBlockK, n0, pol_b);
+        if (j < n_i8) {
+          mbar_arrive_expect_tx(&full[s], a_bytes + b_bytes);
+          tma_load_2d(a_slot(s), &tm_a, &full[s], (kb_begin + j) * kBlockK, m0, pol_a);
+          issue_b(j, s, pol_b);
         } else {
-          const int kb = kb_begin + (j - n_out);
-          if (!W4) {
-            mbar_arrive_expect_tx(&full[s], C::kA + C::kB);
-            tma_load_2d(sA, &tm_a, &full[s], kb * kBlockK, m0, pol_a);
-            tma_load_2d(sB, &tm_b, &full[s], kb * kBlockK, n0, pol_b);
-          } else {
-            mbar_arrive_expect_tx(&full[s], C::kA + C::kP + BN * 4);
-            tma_load_2d(sA, &tm_a, &full[s], kb * kBlockK, m0, pol_a);
-            tma_load_2d(sP, &tm_b, &full[s], kb * (kBlockK / 2), n0, pol_b);
-            tma_load_2d(sG, &tm_g, &full[s], n0, kb, pol_b);
-          }
+          const int o = j - n_i8;
+          mbar_arrive_expect_tx(&full[s], a_bytes + C::kB);
+          tma_load_2d(a_slot(s), &tm_xo, &full[s], o * kOutBlockK, m0, pol_a);
+          tma_load_2d(b_slot(s), &tm_wo, &full[s], o * kOutBlockK, n0, pol_b);
         }
         issued = j + 1;
       }
@@ -195,26 +281,28 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
       constexpr uint32_t kIdF16 = idesc_f16_f32(kTileM, BN);
       const uint32_t t_i32 = tmem_base;
       const uint32_t t_f32 = tmem_base + BN;
+      griddep_wait();
+      const int n_out = (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
+      const int njobs = p.debug_stall ? 1 : n_i8 + n_out;
       int consumed = 0;
       for (int j = 0; j < njobs; ++j) {
-        const int s = j % C::kStages;
-        const uint32_t ph = (j / C::kStages) & 1;
+        const int s = j % stages;
+        const uint32_t ph = (j / stages) & 1;
         if (!mbar_wait(W4 ? &ready[s] : &full[s], ph, p.wait_limit_ns)) {
           fail(s_err, p.status);
           break;
         }
         tc_fence_after();
-        const uint32_t a_addr = smem_u32(ring + s * C::kStage);
-        const uint64_t ad = sw128_kmajor_desc(a_addr);
-        const uint64_t bd = sw128_kmajor_desc(a_addr + C::kA);
-        if (j < n_out) {
+        const uint64_t ad = sw128_kmajor_desc(smem_u32(a_slot(s)));
+        const uint64_t bd = sw128_kmajor_desc(smem_u32(b_slot(s)));
+        if (j < n_i8) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_f16(t_f32, ad + 2 * k, bd + 2 * k, kIdF16, (j > 0 || k > 0) ? 1u : 0u);
+            mma_i8(t_i32, ad + 2 * k, bd + 2 * k, kIdI8, (j > 0 || k > 0) ? 1u : 0u);
         } else {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_i8(t_i32, ad + 2 * k, bd + 2 * k, kIdI8, (j > n_out || k > 0) ? 1u : 0u);
+            mma_f16(t_f32, ad + 2 * k, bd + 2 * k, kIdF16, (j > n_i8 || k > 0) ? 1u : 0u);
         }
         mma_commit(&empty[s]);
         consumed = j + 1;
@@ -222,42 +310,57 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
       mma_commit(accum_full);
       s_misc[2] = consumed;
     }
+  } else if ((warp == 2 || warp == 3) && !RAW) {
+    // ------------------------------------ token scales of the tile, early
+    griddep_wait();
+    for (int i = threadIdx.x - 64; i < kTileM; i += 64)
+      s_sx[i] = m0 + i < p.M ? p.s_x[m0 + i] : 0.f;
   } else if (W4 && warp >= 4) {
     // ------------------------------------------- 4-bit -> INT8 expansion
+    // Thread -> one weight row, so the row's (s2, z2) constants are decoded
+    // once per K block.
+    constexpr int kCpt = W4 ? BN * 4 / C::kExpandThreads : 1;  // 16-byte chunks per thread
     const int et = threadIdx.x - 128;
+    const int row = et % BN;
+    const int c0 = W4 ? (et / BN) * kCpt : 0;
+    griddep_wait();
+    const int n_out = (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
+    const int njobs = p.debug_stall ? 0 : n_i8 + n_out;
     for (int j = 0; j < njobs; ++j) {
-      const int s = j % C::kStages;
-      const uint32_t ph = (j / C::kStages) & 1;
+      const int s = j % stages;
+      const uint32_t ph = (j / stages) & 1;
       if (!mbar_wait(&full[s], ph, p.wait_limit_ns)) {
         fail(s_err, p.status);
         break;
       }
-      if (j >= n_out) {
-        uint8_t *sB = ring + s * C::kStage + C::kA;
+      if (j < n_i8) {
+        uint8_t *sB = b_slot(s);
         const uint8_t *sP = sB + C::kB;
-        const uint32_t *sG = reinterpret_cast<const uint32_t *>(sP + C::kP);
-#pragma unroll 2
-        for (int t = et; t < BN * 4; t += 128) {
-          const int row = t >> 2, c = t & 3;
-          const uint4 pk = *reinterpret_cast<const uint4 *>(sP + row * 64 + c * 16);
-          const uint32_t g = sG[row];
-          const uint32_t s2 = static_cast<uint32_t>(__half2float(__ushort_as_half(
-              static_cast<unsigned short>(g & 0xFFFFu))));
-          const uint32_t z2 = static_cast<uint32_t>(__half2float(__ushort_as_half(
-              static_cast<unsigned short>(g >> 16))));
-          const uint32_t cst = (128u - z2 * s2) * 0x01010101u;
+        const uint32_t g = reinterpret_cast<const uint32_t *>(sP + C::kP)[row];
+        const uint32_t s2 = static_cast<uint32_t>(__half2float(__ushort_as_half(
+            static_cast<unsigned short>(g & 0xFFFFu))));
+        const uint32_t z2 = static_cast<uint32_t>(__half2float(__ushort_as_half(
+            static_cast<unsigned short>(g >> 16))));
+        const uint32_t cst = (128u - z2 * s2) * 0x01010101u;
+        const int psw = (row >> 1) & 3, osw = row & 7;
+        uint4 pk[kCpt];
+#pragma unroll
+        for (int i = 0; i < kCpt; ++i)
+          pk[i] = *reinterpret_cast<const uint4 *>(sP + row * 64 + (((c0 + i) ^ psw) << 4));
+#pragma unroll
+        for (int i = 0; i < kCpt; ++i) {
+          const int c = c0 + i;
           uint4 o0, o1;
-          o0.x = expand4(pk.x & 0x0F0F0F0Fu, s2, cst);
-          o0.y = expand4((pk.x >> 4) & 0x0F0F0F0Fu, s2, cst);
-          o0.z = expand4(pk.y & 0x0F0F0F0Fu, s2, cst);
-          o0.w = expand4((pk.y >> 4) & 0x0F0F0F0Fu, s2, cst);
-          o1.x = expand4(pk.z & 0x0F0F0F0Fu, s2, cst);
-          o1.y = expand4((pk.z >> 4) & 0x0F0F0F0Fu, s2, cst);
-          o1.z = expand4(pk.w & 0x0F0F0F0Fu, s2, cst);
-          o1.w = expand4((pk.w >> 4) & 0x0F0F0F0Fu, s2, cst);
-          const int sw = row & 7;
-          *reinterpret_cast<uint4 *>(sB + row * 128 + (((2 * c) ^ sw) << 4)) = o0;
-          *reinterpret_cast<uint4 *>(sB + row * 128 + (((2 * c + 1) ^ sw) << 4)) = o1;
+          o0.x = expand4(pk[i].x & 0x0F0F0F0Fu, s2, cst);
+          o0.y = expand4((pk[i].x >> 4) & 0x0F0F0F0Fu, s2, cst);
+          o0.z = expand4(pk[i].y & 0x0F0F0F0Fu, s2, cst);
+          o0.w = expand4((pk[i].y >> 4) & 0x0F0F0F0Fu, s2, cst);
+          o1.x = expand4(pk[i].z & 0x0F0F0F0Fu, s2, cst);
+          o1.y = expand4((pk[i].z >> 4) & 0x0F0F0F0Fu, s2, cst);
+          o1.z = expand4(pk[i].w & 0x0F0F0F0Fu, s2, cst);
+          o1.w = expand4((pk[i].w >> 4) & 0x0F0F0F0Fu, s2, cst);
+          *reinterpret_cast<uint4 *>(sB + row * 128 + (((2 * c) ^ osw) << 4)) = o0;
+          *reinterpret_cast<uint4 *>(sB + row * 128 + (((2 * c + 1) ^ osw) << 4)) = o1;
         }
         fence_proxy_async_smem();
       }
@@ -267,6 +370,9 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
   __syncwarp();
 
   // ---------------------------------------------------------------- epilogue
+  griddep_wait();
+  const int any_out = outliers_present(p, RAW);
+  const bool do_out = any_out && rank == 0;
   if (warp < 4) {
     if (!mbar_wait(accum_full, 0, p.wait_limit_ns)) fail(s_err, p.status);
     tc_fence_after();
@@ -279,7 +385,7 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
     if (warp < 4 && !failed) {
       const int row = warp * 32 + lane;
       const int m = m0 + row;
-      const float sx = (!RAW && m < p.M) ? p.s_x[m] : 0.f;
+      const float sx = RAW ? 0.f : s_sx[row];
 #pragma unroll 1
       for (int c = 0; c < BN / 32; ++c) {
         const int n = n0 + c * 32;
@@ -298,11 +404,11 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
                                  static_cast<int>(acc[4 * i + 2]),
                                  static_cast<int>(acc[4 * i + 3]));
           } else {
-            const float4 *sw4 = reinterpret_cast<const float4 *>(p.s_w + n);
+            const float4 *sw4 = reinterpret_cast<const float4 *>(s_sw + c * 32);
             uint32_t h[16];
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
-              const float4 w = __ldg(sw4 + i);
+              const float4 w = sw4[i];
               const float wv[4] = {w.x, w.y, w.z, w.w};
               float y[4];
 #pragma unroll
@@ -330,8 +436,8 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
   } else {
     // ------------------------------------ K split: reduce across the cluster
     int32_t *pbuf = reinterpret_cast<int32_t *>(ring);
-    float *obuf = reinterpret_cast<float *>(ring + kTileM * C::kPitch * 4);
-    const int rows_valid = min(kTileM, p.M - m0);
+    float *obuf = reinterpret_cast<float *>(ring + C::kRedRows * C::kPitch * 4);
+    const int rows_valid = min(C::kRedRows, p.M - m0);
     const uint32_t my_rank = cluster_ctarank();
     // this CTA reduces columns [c_begin, c_end) of each 128-column chunk
     const int c_begin = static_cast<int>(my_rank) * (C::kCW / 4) / S * 4;
@@ -376,28 +482,32 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
           if (n >= p.N) continue;
           const int m = m0 + row;
           const uint32_t off = smem_u32(pbuf + row * C::kPitch + col);
+          // issue every peer's load before summing, so their latencies overlap
+          int4 part[C::kMaxStages];
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            if (q < S) part[q] = ld_dsmem_v4(mapa_shared(off, static_cast<uint32_t>(q)));
+          int4 oi = make_int4(0, 0, 0, 0);
+          if (!RAW && any_out)
+            oi = ld_dsmem_v4(mapa_shared(smem_u32(obuf + row * C::kPitch + col), 0u));
           int4 sum = make_int4(0, 0, 0, 0);
-          for (int q = 0; q < S; ++q) {
-            const int4 v = ld_dsmem_v4(mapa_shared(off, static_cast<uint32_t>(q)));
-            sum.x += v.x;
-            sum.y += v.y;
-            sum.z += v.z;
-            sum.w += v.w;
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (q < S) {
+              sum.x += part[q].x;
+              sum.y += part[q].y;
+              sum.z += part[q].z;
+              sum.w += part[q].w;
+            }
           }
           if (RAW) {
             *reinterpret_cast<int4 *>(static_cast<int32_t *>(p.Y) + static_cast<size_t>(m) * p.ldy +
                                       n) = sum;
           } else {
-            float ov[4] = {0.f, 0.f, 0.f, 0.f};
-            if (any_out) {
-              const int4 oi = ld_dsmem_v4(mapa_shared(smem_u32(obuf + row * C::kPitch + col), 0u));
-              ov[0] = __int_as_float(oi.x);
-              ov[1] = __int_as_float(oi.y);
-              ov[2] = __int_as_float(oi.z);
-              ov[3] = __int_as_float(oi.w);
-            }
-            const float sx = p.s_x[m];
-            const float4 w = __ldg(reinterpret_cast<const float4 *>(p.s_w + n));
+            const float ov[4] = {__int_as_float(oi.x), __int_as_float(oi.y), __int_as_float(oi.z),
+                                 __int_as_float(oi.w)};
+            const float sx = s_sx[row];
+            const float4 w = *reinterpret_cast<const float4 *>(s_sw + r * C::kCW + col);
             const int si[4] = {sum.x, sum.y, sum.z, sum.w};
             const float wv[4] = {w.x, w.y, w.z, w.w};
             float y[4];
@@ -427,7 +537,7 @@ __global__ void __launch_bounds__(Cfg<BN, W4>::kThreads, 1)
     // Let any tile copy still in flight land before the CTA's shared memory
     // is released: wait (bounded) for every load issued but never consumed.
     for (int j = s_misc[2]; j < s_misc[3]; ++j)
-      mbar_wait(&full[j % C::kStages], (j / C::kStages) & 1, p.wait_limit_ns);
+      mbar_wait(&full[j % stages], (j / stages) & 1, p.wait_limit_ns);
   }
   if (warp == 1) {
     tc_fence_after();
@@ -480,38 +590,76 @@ cudaError_t ensure_smem(K kernel, int bytes, std::atomic<uint64_t> &done_mask) {
   const uint64_t bit = 1ull << (dev & 63);
   if (done_mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
   e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  // all of the unified L1/shared array as shared memory, so that two small-M
+  // CTAs (about 106 KB each) fit on one SM
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
+                             cudaSharedmemCarveoutMaxShared);
   if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_acq_rel);
   return e;
 }
 
-template <int BN, bool W4, bool RAW>
+// Pipeline geometry of a launch: stage count, A slot size, dynamic smem.
+// Full-size variants use 128-row A slots and a fixed depth; the small-M
+// variant sizes its A slots to the token rows and takes as many stages as fit
+// in half an SM's shared memory (so a CTA of the next kernel fits beside it).
+struct Geometry {
+  int stages, a_stride, smem;
+};
+
+template <int BN, bool W4, bool SM>
+Geometry geometry(int M, int split) {
+  using C = Cfg<BN, W4, SM>;
+  Geometry g{};
+  if (!SM) {
+    g.stages = C::kStages;
+    g.a_stride = kTileM * kBlockK;
+  } else {
+    const int a_rows = M >= 64 ? 64 : (M + 7) / 8 * 8;
+    g.a_stride = a_rows * kBlockK;
+    const int budget = 233472 / 2 - 1024 - C::kExtra - 1024;  // half an SM, minus reserve
+    g.stages = budget / (g.a_stride + C::kBStage);
+    if (g.stages > C::kMaxStages) g.stages = C::kMaxStages;
+    while (split > 1 && g.stages < C::kMaxStages &&
+           C::ring_bytes(g.stages, g.a_stride) < C::kRedBytes)
+      ++g.stages;
+  }
+  g.smem = C::smem_bytes(g.stages, g.a_stride);
+  return g;
+}
+
+template <int BN, bool W4, bool SM>
+constexpr int max_smem() {
+  using C = Cfg<BN, W4, SM>;
+  return SM ? 233472 / 2 - 1024 : C::smem_bytes(C::kStages, kTileM * kBlockK);
+}
+
+template <int BN, bool W4, bool SM, bool RAW>
 cudaError_t launch_variant(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
                            const char **why) {
-  using C = Cfg<BN, W4>;
+  using C = Cfg<BN, W4, SM>;
+  static_assert(max_smem<BN, W4, SM>() <= 232448, "shared memory budget");
   static std::atomic<uint64_t> smem_done{0};
-  auto kernel = mixq_gemm_kernel<BN, W4, RAW>;
-  cudaError_t e = ensure_smem(kernel, C::kSmem, smem_done);
+  auto kernel = mixq_gemm_kernel<BN, W4, SM, RAW>;
+  cudaError_t e = ensure_smem(kernel, max_smem<BN, W4, SM>(), smem_done);
   if (e != cudaSuccess) return e;
+  const Geometry geo = geometry<BN, W4, SM>(a.M, plan.split);
+  if (geo.smem > max_smem<BN, W4, SM>() || geo.stages < 2 ||
+      (plan.split > 1 && C::ring_bytes(geo.stages, geo.a_stride) < C::kRedBytes)) {
+    *why = "no pipeline geometry fits the shared-memory budget";
+    return cudaErrorInvalidValue;
+  }
 
   const int kp = k_out_pad(a.K_out);
-  alignas(64) CUtensorMap tm_a, tm_b, tm_g, tm_xo, tm_wo;
-  memset(&tm_g, 0, sizeof tm_g);
+  const int a_rows = a.M >= kTileM ? kTileM : (a.M + 7) / 8 * 8;
+  alignas(64) CUtensorMap tm_a, tm_xo, tm_wo;
   memset(&tm_xo, 0, sizeof tm_xo);
   memset(&tm_wo, 0, sizeof tm_wo);
   bool ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Xq, a.K, a.M, a.K, kBlockK,
-                     kTileM, CU_TENSOR_MAP_SWIZZLE_128B);
-  if (!W4) {
-    ok = ok && make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Wq, a.K, a.N, a.K, kBlockK,
-                        BN, CU_TENSOR_MAP_SWIZZLE_128B);
-  } else {
-    ok = ok && make_map(&tm_b, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Wq, a.K / 2, a.N, a.K / 2,
-                        kBlockK / 2, BN, CU_TENSOR_MAP_SWIZZLE_NONE);
-    ok = ok && make_map(&tm_g, CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, a.grp, a.N, a.K / kGroup,
-                        static_cast<uint64_t>(a.N) * 4, BN, 1, CU_TENSOR_MAP_SWIZZLE_NONE);
-  }
-  if (!RAW && kp > 0) {
+                     a_rows, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (a.epi != Epi::kRawI32 && kp > 0) {
     ok = ok && make_map(&tm_xo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.X_out, kp, a.M,
-                        static_cast<uint64_t>(kp) * 2, kOutBlockK, kTileM,
+                        static_cast<uint64_t>(kp) * 2, kOutBlockK, a_rows,
                         CU_TENSOR_MAP_SWIZZLE_128B);
     ok = ok && make_map(&tm_wo, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.W_out, kp, a.N,
                         static_cast<uint64_t>(kp) * 2, kOutBlockK, BN,
@@ -527,6 +675,11 @@ cudaError_t launch_variant(const GemmArgs &a, const GemmPlan &plan, cudaStream_t
   kp_.N = a.N;
   kp_.K = a.K;
   kp_.K_out_pad = RAW ? 0 : kp;
+  kp_.a_rows = a_rows;
+  kp_.a_stride = geo.a_stride;
+  kp_.stages = geo.stages;
+  kp_.wq = static_cast<const uint8_t *>(a.Wq);
+  kp_.grp = static_cast<const uint8_t *>(a.grp);
   kp_.s_x = a.s_x;
   kp_.s_w = a.s_w;
   kp_.flags = a.flags;
@@ -542,50 +695,156 @@ cudaError_t launch_variant(const GemmArgs &a, const GemmPlan &plan, cudaStream_t
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(m_tiles, n_tiles, plan.split);
   cfg.blockDim = dim3(C::kThreads, 1, 1);
-  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.dynamicSmemBytes = geo.smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 1;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = plan.split;
+  // programmatic dependent launch: the CTAs may start (and stream weights)
+  // while the preceding kernel in the stream finishes; they wait for it with
+  // griddepcontrol.wait before touching its outputs
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_xo, tm_wo, kp_);
+}
+
+template <int BN, bool W4, bool SM>
+int max_active_clusters_variant(int split) {
+  using C = Cfg<BN, W4, SM>;
+  static std::atomic<uint64_t> smem_done{0};
+  auto kernel = mixq_gemm_kernel<BN, W4, SM, false>;
+  if (ensure_smem(kernel, max_smem<BN, W4, SM>(), smem_done) != cudaSuccess) return -1;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(1, 1, split);
+  cfg.blockDim = dim3(C::kThreads, 1, 1);
+  cfg.dynamicSmemBytes = geometry<BN, W4, SM>(SM ? 16 : 4096, split).smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 1;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = split;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_b, tm_g, tm_xo, tm_wo, kp_);
+  int n = -1;
+  if (cudaOccupancyMaxActiveClusters(&n, kernel, &cfg) != cudaSuccess) return -1;
+  return n;
 }
 
 }  // namespace
 
-GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms) {
-  // Time model (microseconds).  Compute: waves of CTAs (one per SM), each
-  // running its K range at one 128 x BN x 128 INT8 MMA stage per
-  // 0.28 us * BN/256, plus a fixed prologue/epilogue and the cluster
-  // reduction when K is split.  Memory: the bytes that must come from HBM at
-  // least once (weights, activations, output) at the smaller of the HBM
-  // rate and what the active SMs can pull (~60 GB/s each).  The plan with
-  // the smaller max(compute, memory) wins; ties keep fewer CTAs.
-  GemmPlan best{256, 1, 0};
+const ClusterLimits *device_cluster_limits(int mode) {
+  static ClusterLimits table[64][2];
+  static std::atomic<int> ready[64][2];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  const int md = mode == 1 ? 1 : 0;
+  if (ready[dev][md].load(std::memory_order_acquire)) return &table[dev][md];
+  static std::mutex mu;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ready[dev][md].load(std::memory_order_acquire)) {
+    ClusterLimits &t = table[dev][md];
+    for (int small = 0; small < 2; ++small)
+      for (int wide = 0; wide < 2; ++wide)
+        for (int s = 0; s <= 8; ++s)
+          t.max_active[small][wide][s] =
+              (s == 0 || (small && wide)) ? 0
+                                          : gemm_max_active_clusters(md, wide ? 256 : 128, s, small);
+    ready[dev][md].store(1, std::memory_order_release);
+  }
+  return &table[dev][md];
+}
+
+int gemm_max_active_clusters(int mode, int bn, int split, int small_m) {
+  if (small_m) {
+    if (bn == 32) return mode == 1 ? max_active_clusters_variant<32, true, true>(split)
+                                   : max_active_clusters_variant<32, false, true>(split);
+    if (bn == 64) return mode == 1 ? max_active_clusters_variant<64, true, true>(split)
+                                   : max_active_clusters_variant<64, false, true>(split);
+    if (bn != 128) return -1;
+    return mode == 1 ? max_active_clusters_variant<128, true, true>(split)
+                     : max_active_clusters_variant<128, false, true>(split);
+  }
+  if (bn == 256) return mode == 1 ? max_active_clusters_variant<256, true, false>(split)
+                                  : max_active_clusters_variant<256, false, false>(split);
+  return mode == 1 ? max_active_clusters_variant<128, true, false>(split)
+                   : max_active_clusters_variant<128, false, false>(split);
+}
+
+int estimate_max_active_clusters(int num_sms, int ctas_per_sm, int split) {
+  // SMs come in GPCs of about 18 and a cluster lives inside one GPC.
+  const int gpcs = (num_sms + 9) / 18 > 0 ? (num_sms + 9) / 18 : 1;
+  const int per_gpc = num_sms / gpcs;
+  return gpcs * ((per_gpc * ctas_per_sm) / split);
+}
+
+GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimits *limits) {
+  if (M <= 64) {
+    // Decode-sized M is latency bound: a CTA streams one 16 KB weight stage
+    // per ~0.4 us whatever the tile width (measured), so what matters is how
+    // many CTAs stream at once.  128-wide tiles, K split into the smallest
+    // cluster that brings the CTA count to about one per SM (never past
+    // 1.25 per SM, never past one wave of clusters).
+    const int KB = K / kBlockK;
+    const int n_tiles = N / 128;
+    int best_s = 1;
+    for (int s = 1; s <= 8 && s <= KB; ++s) {
+      const int ctas = n_tiles * s;
+      const int clusters_per_wave =
+          limits ? limits->max_active[1][0][s] : estimate_max_active_clusters(num_sms, 2, s);
+      if (ctas > num_sms + num_sms / 4 || n_tiles > clusters_per_wave) break;
+      best_s = s;
+      if (ctas * 5 >= num_sms * 4) break;
+    }
+    return GemmPlan{128, best_s, n_tiles * best_s, 1};
+  }
+  // Time model (microseconds at ~1.9 GHz).  CTAs run in waves; a wave holds
+  // at most max_active(split) clusters of `split` CTAs (one CTA per SM; two for
+  // the small-M variants).  A K block costs a CTA the larger of its MMA cycles
+  // (8192 INT8 MACs per cycle) and its shared-memory cycles (the MMA reads all
+  // 128 A rows plus the BN B rows at 128 B per cycle) -- narrow tiles are
+  // shared-memory bound.  Fixed cost per CTA: prologue/epilogue, plus the
+  // cluster reduction (which waits for the slowest peer) when K is split.
+  // Memory: the bytes that must come from HBM at least once (weights,
+  // activations, output) at the HBM rate.  Cost = max(compute, memory); ties
+  // keep fewer CTAs.
+  GemmPlan best{256, 1, 0, 0};
   double best_cost = 1e300;
   const int m_tiles = (M + kTileM - 1) / kTileM;
   const int KB = K / kBlockK;
   const double w_bytes = (mode == 1 ? 0.5 + 4.0 / kGroup : 1.0) * static_cast<double>(N) * K;
   const double unique_bytes = w_bytes + static_cast<double>(M) * K + 2.0 * M * N;
-  const int bns[2] = {256, 128};
-  for (int bn : bns) {
-    const int n_tiles = (N + bn - 1) / bn;
+  struct Variant { int bn, small; };
+  const Variant variants[2] = {{256, 0}, {128, 0}};
+  for (const Variant v : variants) {
+    const int wide = v.bn == 256 ? 1 : 0;
+    const double mma_cyc = 4.0 * 128 * v.bn * 32 / 8192.0;
+    const double smem_cyc = (16384.0 + v.bn * 128.0) / 128.0;
+    const double t_kb = (mma_cyc > smem_cyc ? mma_cyc : smem_cyc) / 1900.0;
+    const int n_tiles = (N + v.bn - 1) / v.bn;
     for (int s = 1; s <= 8 && s <= KB; ++s) {
+      int clusters_per_wave = 0;
+      if (limits && v.bn >= 128)
+        clusters_per_wave = limits->max_active[v.small][wide][s];
+      else if (limits && limits->max_active[1][0][s] > 0)
+        clusters_per_wave = limits->max_active[1][0][s];  // narrow tiles: same footprint class
+      else
+        clusters_per_wave = estimate_max_active_clusters(num_sms, v.small ? 2 : 1, s);
+      if (clusters_per_wave <= 0) continue;
+      const long long slots = static_cast<long long>(clusters_per_wave) * s;
       const long long ctas = static_cast<long long>(m_tiles) * n_tiles * s;
-      const long long waves = (ctas + num_sms - 1) / num_sms;
+      const long long waves = (ctas + slots - 1) / slots;
       const int kb_per = (KB + s - 1) / s;
-      const double fixed = 1.0 + (s > 1 ? 0.3 + 0.05 * s : 0.0);
-      const double compute = waves * (kb_per * 0.28 * (bn / 256.0) + fixed);
-      const double active = static_cast<double>(ctas < num_sms ? ctas : num_sms);
-      const double bw = active * 60e3 < 6.5e6 ? active * 60e3 : 6.5e6;  // bytes per us
-      const double memory = unique_bytes / bw + fixed;
+      const double fixed = 1.5 + (s > 1 ? 1.5 + 0.05 * s : 0.0);
+      const double compute = waves * (kb_per * t_kb + fixed);
+      const double memory = unique_bytes / 6.5e6 + fixed;
       const double cost = compute > memory ? compute : memory;
       if (cost < best_cost * (1 - 1e-6)) {
         best_cost = cost;
-        best = GemmPlan{bn, s, static_cast<int>(ctas)};
+        best = GemmPlan{v.bn, s, static_cast<int>(ctas), v.small};
       }
     }
   }
@@ -596,16 +855,19 @@ cudaError_t launch_gemm(const GemmArgs &a, const GemmPlan &plan, cudaStream_t st
                         const char **why) {
   const bool w4 = a.mode == 1;
   const bool raw = a.epi == Epi::kRawI32;
-  if (plan.bn == 256) {
-    if (w4) return raw ? launch_variant<256, true, true>(a, plan, stream, why)
-                       : launch_variant<256, true, false>(a, plan, stream, why);
-    return raw ? launch_variant<256, false, true>(a, plan, stream, why)
-               : launch_variant<256, false, false>(a, plan, stream, why);
+#define MIXQ_DISPATCH(BN_, SM_)                                                      \
+  if (w4) return raw ? launch_variant<BN_, true, SM_, true>(a, plan, stream, why)   \
+                     : launch_variant<BN_, true, SM_, false>(a, plan, stream, why); \
+  return raw ? launch_variant<BN_, false, SM_, true>(a, plan, stream, why)          \
+             : launch_variant<BN_, false, SM_, false>(a, plan, stream, why);
+  if (plan.small_m) {
+    if (plan.bn == 32) { MIXQ_DISPATCH(32, true) }
+    if (plan.bn == 64) { MIXQ_DISPATCH(64, true) }
+    MIXQ_DISPATCH(128, true)
   }
-  if (w4) return raw ? launch_variant<128, true, true>(a, plan, stream, why)
-                     : launch_variant<128, true, false>(a, plan, stream, why);
-  return raw ? launch_variant<128, false, true>(a, plan, stream, why)
-             : launch_variant<128, false, false>(a, plan, stream, why);
+  if (plan.bn == 256) { MIXQ_DISPATCH(256, false) }
+  MIXQ_DISPATCH(128, false)
+#undef MIXQ_DISPATCH
 }
 
 }  // namespace mixq

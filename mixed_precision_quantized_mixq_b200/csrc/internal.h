@@ -18,6 +18,7 @@ constexpr int kTileM = 128;     // output tile rows (tcgen05 M)
 inline int k_out_pad(int k_out) { return (k_out + 63) / 64 * 64; }
 
 // ---------------------------------------------------------------- quantize
+int quantize_max_k();  // largest K the quantize kernel holds in registers
 cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx,
                                 int K_out, float threshold, int8_t *Xq, float *s_x, void *X_out,
                                 uint32_t *bitmap, int32_t *flags, int32_t *status,
@@ -27,17 +28,27 @@ cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int3
 cudaError_t launch_prepack(int mode, const void *W, int N, int K, const int32_t *idx, int K_out,
                            void *Wq, float *s_w, void *grp, void *W_out, int32_t *status,
                            cudaStream_t stream);
+cudaError_t launch_unpack_w8(int N, int K, const void *Wq, int8_t *out, cudaStream_t stream);
 cudaError_t launch_unpack_w4(int N, int K, const void *Wq4, const void *grp, uint8_t *q,
                              uint8_t *s2, uint8_t *z2, cudaStream_t stream);
 
 // -------------------------------------------------------------------- gemm
 struct GemmPlan {
-  int bn;     // output tile width (128 or 256)
-  int split;  // K split = cluster size along z (1..8)
-  int ctas;   // total CTAs launched
+  int bn;       // output tile width (128 or 256)
+  int split;    // K split = cluster size along z (1..8)
+  int ctas;     // total CTAs launched
+  int small_m;  // M <= 64 kernel variant (two CTAs per SM), bn == 128 only
 };
 
-GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms);
+// How many clusters of `split` CTAs run at once, per [small-M][bn == 256][split].
+struct ClusterLimits {
+  int max_active[2][2][9];
+};
+// limits == nullptr: estimate from num_sms (GPCs of about 18 SMs).
+GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimits *limits);
+int estimate_max_active_clusters(int num_sms, int ctas_per_sm, int split);
+int gemm_max_active_clusters(int mode, int bn, int split, int small_m);  // -1 on error
+const ClusterLimits *device_cluster_limits(int mode);  // current device, cached; may be null
 
 enum class Epi { kMixed = 0, kRawI32 = 1 };
 

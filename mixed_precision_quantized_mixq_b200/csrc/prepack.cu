@@ -9,10 +9,23 @@
 // "MixLLM: Ein neuer Ansatz"): the INT8 codes are quantized again per group of
 // 128 along K with an integer scale s2 and zero z2 chosen so that the
 // effective weight (q - z2) * s2 always fits int8; the GEMM mainloop rebuilds
-// it with one integer multiply-add per four codes.  Packed layout: byte
-// (n, 64g + b) holds q[n, 128g + 8(b>>2) + (b&3)] in its low nibble and the
-// code four positions later in its high nibble, so a 32-bit word splits into
-// two words of four consecutive codes with one mask and one shift.
+// it with one integer multiply-add per four codes.
+//
+// Both code layouts are reordered for the GEMM (QServe notes, "compute-aware
+// weight reordering": the layout is chosen so the kernel's loads need no
+// address arithmetic): the weights are cut into tiles of 128 output channels
+// x 128 K, stored tile after tile (channel tile major, K tile minor), each
+// tile one contiguous block that a single bulk copy moves into shared memory
+// exactly as the tensor core (W8) or the expansion warps (W4) read it.
+//   W8 tile (16 KB): row r at r*128; the 16-byte chunk holding K offsets
+//     16j..16j+15 sits at chunk position j ^ (r & 7) (the 128-byte swizzle of
+//     a K-major tcgen05 operand).
+//   W4 tile (8 KB): row r at r*64; the 16-byte chunk c (K offsets 32c..32c+31)
+//     sits at chunk position c ^ ((r >> 1) & 3) (conflict-free row reads);
+//     inside a chunk, byte 4w+i holds the code of K offset 32c+8w+i in its low
+//     nibble and that of 32c+8w+4+i in its high nibble, so a 32-bit word
+//     splits into two words of four consecutive codes with one mask and one
+//     shift.
 #include <cuda_fp16.h>
 
 #include "internal.h"
@@ -23,6 +36,21 @@ namespace {
 
 constexpr int kPThreads = 256;
 constexpr int kPWarps = kPThreads / 32;
+
+// Byte offset of W8 code (n, k) in the tiled layout (k a multiple of 8 gives
+// the start of 8 consecutive codes inside one 16-byte chunk).
+__host__ __device__ __forceinline__ size_t w8_offset(int n, int k, int KB) {
+  const size_t tile = static_cast<size_t>(n >> 7) * KB + (k >> 7);
+  const int r = n & 127;
+  return (tile * 128 + r) * 128 + ((((k & 127) >> 4) ^ (r & 7)) << 4) + (k & 15);
+}
+
+// Byte offset of 4-bit chunk c (K offsets 32c..32c+31 of K tile kb) of row n.
+__host__ __device__ __forceinline__ size_t w4_chunk_offset(int n, int kb, int c, int KB) {
+  const size_t tile = static_cast<size_t>(n >> 7) * KB + kb;
+  const int r = n & 127;
+  return (tile * 128 + r) * 64 + ((c ^ ((r >> 1) & 3)) << 4);
+}
 
 __device__ __forceinline__ float warp_max_f(float v) {
 #pragma unroll
@@ -89,7 +117,7 @@ __global__ void __launch_bounds__(kPThreads) prepack_kernel(
       if (kW4) {
         reinterpret_cast<uint2 *>(psm)[v] = make_uint2(word[0], word[1]);
       } else {
-        reinterpret_cast<uint2 *>(static_cast<int8_t *>(Wq) + static_cast<size_t>(n) * K)[v] =
+        *reinterpret_cast<uint2 *>(static_cast<int8_t *>(Wq) + w8_offset(n, v * 8, K / 128)) =
             make_uint2(word[0], word[1]);
       }
     }
@@ -136,11 +164,10 @@ __global__ void __launch_bounds__(kPThreads) prepack_kernel(
               __halves2half2(__int2half_rn(s2), __int2half_rn(z2));
       }
       __syncthreads();
-      // Pack: 4 output bytes (one 32-bit word = 8 codes) per thread and step.
-      uint32_t *dst = reinterpret_cast<uint32_t *>(static_cast<uint8_t *>(Wq) +
-                                                   static_cast<size_t>(n) * (K / 2));
+      // Pack: one 32-bit word (8 codes, k = 8wi .. 8wi+7) per thread and step.
+      uint8_t *dst = static_cast<uint8_t *>(Wq);
       for (int wi = tid; wi < K / 8; wi += kPThreads) {
-        const int8_t *src = psm + wi * 8;  // codes k = 8wi .. 8wi+7
+        const int8_t *src = psm + wi * 8;
         uint32_t word = 0;
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -148,7 +175,8 @@ __global__ void __launch_bounds__(kPThreads) prepack_kernel(
                                 ((static_cast<uint32_t>(src[i + 4]) & 0xFu) << 4);
           word |= byte << (8 * i);
         }
-        dst[wi] = word;
+        const int kb = wi >> 4, c = (wi >> 2) & 3, w = wi & 3;
+        *reinterpret_cast<uint32_t *>(dst + w4_chunk_offset(n, kb, c, K / 128) + 4 * w) = word;
       }
       __syncthreads();
     }
@@ -164,14 +192,24 @@ __global__ void unpack_w4_kernel(int N, int K, const uint8_t *__restrict__ Wq4,
        i += static_cast<size_t>(gridDim.x) * blockDim.x) {
     const int n = static_cast<int>(i / K), k = static_cast<int>(i % K);
     const int g = k / kGroup, r = k % kGroup;
-    const int b = 4 * (r >> 3) + (r & 3);
-    const uint8_t byte = Wq4[static_cast<size_t>(n) * (K / 2) + g * 64 + b];
-    q[i] = (r & 4) ? (byte >> 4) : (byte & 0xF);
+    const int c = r >> 5, w = (r >> 3) & 3, e = r & 7;
+    const uint8_t byte = Wq4[w4_chunk_offset(n, g, c, groups) + 4 * w + (e & 3)];
+    q[i] = (e & 4) ? (byte >> 4) : (byte & 0xF);
     if (r == 0) {
       const float2 sz = __half22float2(grp[static_cast<size_t>(g) * N + n]);
       s2[static_cast<size_t>(n) * groups + g] = static_cast<uint8_t>(sz.x);
       z2[static_cast<size_t>(n) * groups + g] = static_cast<uint8_t>(sz.y);
     }
+  }
+}
+
+__global__ void unpack_w8_kernel(int N, int K, const int8_t *__restrict__ Wq,
+                                 int8_t *__restrict__ out) {
+  const size_t total = static_cast<size_t>(N) * K;
+  for (size_t i = blockIdx.x * static_cast<size_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<size_t>(gridDim.x) * blockDim.x) {
+    const int n = static_cast<int>(i / K), k = static_cast<int>(i % K);
+    out[i] = Wq[w8_offset(n, k, K / 128)];
   }
 }
 
@@ -207,4 +245,12 @@ cudaError_t launch_unpack_w4(int N, int K, const void *Wq4, const void *grp, uin
   return cudaGetLastError();
 }
 
+}  // namespace mixq
+
+namespace mixq {
+cudaError_t launch_unpack_w8(int N, int K, const void *Wq, int8_t *out, cudaStream_t stream) {
+  if (N == 0) return cudaSuccess;
+  unpack_w8_kernel<<<1024, 256, 0, stream>>>(N, K, static_cast<const int8_t *>(Wq), out);
+  return cudaGetLastError();
+}
 }  // namespace mixq

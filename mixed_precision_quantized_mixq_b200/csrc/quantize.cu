@@ -5,10 +5,23 @@
 // MixQ的解决方案: the amax of quantization doubles as the outlier test;
 // Fig. 10 equivalent transformation; Fig. 11 order-preserved outlier matrix).
 //
-// HBM-bound: one read of X (16-byte vector loads, the second pass over a row
-// hits L1), one write of Xq (8-byte stores), K_out_pad fp16 per token of
-// X_out.  One CTA walks token rows with a grid stride; the outlier channel
-// mask lives in shared memory as a bitset built once per CTA.
+// HBM-bound: X is read once with 16-byte vector loads and kept in registers
+// (VPT vectors per thread), Xq is written with 8-byte stores, the outlier
+// channels of a mixed token are scattered straight from registers into X_out
+// (a channel's column is its rank in the sorted outlier list, from a prefix
+// count over the outlier bitset kept in shared memory).  A group of 256
+// threads owns one token at a time; a CTA holds G such groups.
+//
+// Matrix-wide outputs (bitmap, flags):
+//   - one thread-block cluster covers all tokens (decode-sized M): CTAs keep
+//     their detection words and counts in shared memory and the cluster
+//     combines them through distributed shared memory; plain stores, no
+//     atomics and no reset pass;
+//   - otherwise: a 1-block reset kernel zeroes bitmap/flags, CTAs OR/add into
+//     them with atomics, and the last CTA to finish (ticket in flags[2])
+//     counts the detections outside the outlier list.
+// All kernels use programmatic dependent launch: they wait for the preceding
+// grid before their first global memory access.
 #include <cuda_fp16.h>
 
 #include "internal.h"
@@ -17,13 +30,17 @@
 namespace mixq {
 namespace {
 
-constexpr int kQThreads = 256;
-constexpr int kQWarps = kQThreads / 32;
+constexpr int kRowThreads = 256;  // threads per token group
+constexpr int kRowWarps = kRowThreads / 32;
+constexpr int kMaxClusterCtas = 8;
 
 __global__ void reset_detect_kernel(uint32_t *__restrict__ bitmap, int words,
                                     int32_t *__restrict__ flags) {
+  griddep_wait();
   for (int w = threadIdx.x; w < words; w += blockDim.x) bitmap[w] = 0u;
   if (threadIdx.x < 4) flags[threadIdx.x] = 0;
+  __syncthreads();
+  if (threadIdx.x == 0) griddep_launch_dependents();
 }
 
 __device__ __forceinline__ float warp_max(float v) {
@@ -45,49 +62,109 @@ __device__ __forceinline__ uint32_t code8(float x, float inv) {
   return static_cast<uint32_t>(q) & 0xFFu;
 }
 
-__global__ void __launch_bounds__(kQThreads) quantize_act_kernel(
-    const __half *__restrict__ X, int M, int K, int ldx, const int32_t *__restrict__ idx,
-    int K_out, int K_out_pad, float T, int8_t *__restrict__ Xq, float *__restrict__ s_x,
-    __half *__restrict__ X_out, uint32_t *__restrict__ bitmap, int32_t *__restrict__ flags,
-    int32_t *__restrict__ status) {
+struct QArgs {
+  const __half *X;
+  int M, K, ldx;
+  const int32_t *idx;
+  int K_out, K_out_pad;
+  float T;
+  int8_t *Xq;
+  float *s_x;
+  __half *X_out;
+  uint32_t *bitmap;
+  int32_t *flags;
+  int32_t *status;
+  int cluster_mode;  // one cluster covers the whole grid
+};
+
+template <int VPT, int G>
+__global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArgs a) {
   extern __shared__ uint32_t qsm[];
-  const int words = K >> 5;  // K % 128 == 0
-  uint32_t *s_mask = qsm;                                    // outlier channel bitset
-  uint32_t *s_det = qsm + words;                             // channels with |x| > T
-  int32_t *s_idx = reinterpret_cast<int32_t *>(qsm + 2 * words);  // validated idx copy
-  __shared__ float s_red[2][kQWarps];
-  __shared__ int s_bad, s_last, s_cnt[kQWarps];
+  const int words = a.K >> 5;  // K % 128 == 0
+  uint32_t *s_mask = qsm;               // outlier channel bitset
+  uint32_t *s_det = qsm + words;        // channels with |x| > T seen by this CTA
+  uint32_t *s_rank = qsm + 2 * words;   // outlier channels in words before w
+  __shared__ float s_red[G][2][kRowWarps];
+  __shared__ int s_bad, s_last, s_part[2], s_cnt[G * kRowWarps];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  for (int w = tid; w < words; w += kQThreads) {
+  const int g = tid / kRowThreads, gt = tid % kRowThreads, gw = gt >> 5;
+  const int nvec = a.K >> 3;  // 8 fp16 per 16-byte vector
+  const int row_stride = gridDim.x * G;
+
+  griddep_wait();
+  // Start this group's first token load before the outlier bitset is built
+  // so the two latencies overlap.
+  int m = blockIdx.x * G + g;
+  uint4 v[VPT];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int vi = gt + i * kRowThreads;
+    v[i] = (m < a.M && vi < nvec)
+               ? __ldg(reinterpret_cast<const uint4 *>(a.X + static_cast<size_t>(m) * a.ldx) + vi)
+               : make_uint4(0u, 0u, 0u, 0u);
+  }
+  for (int w = tid; w < words; w += blockDim.x) {
     s_mask[w] = 0u;
     s_det[w] = 0u;
   }
   if (tid == 0) s_bad = 0;
   __syncthreads();
-  for (int j = tid; j < K_out; j += kQThreads) {
-    int c = idx[j];
-    const bool ok = c >= 0 && c < K && (j == 0 || idx[j - 1] < c);
-    if (!ok) {
-      s_bad = 1;
-      c = -1;
-    }
-    s_idx[j] = c;
-    if (c >= 0) atomicOr(&s_mask[c >> 5], 1u << (c & 31));
+  for (int j = tid; j < a.K_out; j += blockDim.x) {
+    const int c = a.idx[j];
+    const bool ok = c >= 0 && c < a.K && (j == 0 || a.idx[j - 1] < c);
+    if (!ok) s_bad = 1;
+    else atomicOr(&s_mask[c >> 5], 1u << (c & 31));
   }
   __syncthreads();
-  if (s_bad && tid == 0 && blockIdx.x == 0) record_error(status, kErrInvalidArg);
+  if (warp == 0) {  // exclusive prefix count of outlier channels per bitset word
+    const int per = (words + 31) / 32;
+    const int w0 = lane * per;
+    int local = 0;
+    for (int w = w0; w < w0 + per && w < words; ++w) local += __popc(s_mask[w]);
+    int incl = local;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int t = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += t;
+    }
+    int run = incl - local;
+    for (int w = w0; w < w0 + per && w < words; ++w) {
+      s_rank[w] = static_cast<uint32_t>(run);
+      run += __popc(s_mask[w]);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {
+    if (s_bad) record_error(a.status, kErrInvalidArg);
+    griddep_launch_dependents();
+  }
 
-  const int nvec = K >> 3;  // 8 fp16 per 16-byte vector
+  // The group's next token is loaded while this one is processed (when the
+  // two rows fit in registers).
+  constexpr bool kPrefetch = VPT <= 8;
+  constexpr int kVn = kPrefetch ? VPT : 1;
+  auto load_row = [&](int row, uint4 *dst, int count) {
+#pragma unroll
+    for (int i = 0; i < count; ++i) {
+      const int vi = gt + i * kRowThreads;
+      dst[i] = (row < a.M && vi < nvec)
+                   ? __ldg(reinterpret_cast<const uint4 *>(a.X + static_cast<size_t>(row) * a.ldx) +
+                           vi)
+                   : make_uint4(0u, 0u, 0u, 0u);
+    }
+  };
   int mixed_rows = 0;
-  for (int m = blockIdx.x; m < M; m += gridDim.x) {
-    const uint4 *xr = reinterpret_cast<const uint4 *>(X + static_cast<size_t>(m) * ldx);
+  for (; m < a.M; m += row_stride) {
+    uint4 vn[kVn];
+    if (kPrefetch) load_row(m + row_stride, vn, kVn);
     float aI = 0.f, aN = 0.f;
-    for (int v = tid; v < nvec; v += kQThreads) {
-      const uint4 raw = __ldg(xr + v);
-      const int k0 = v << 3;
-      const uint32_t mb = (s_mask[k0 >> 5] >> (k0 & 31)) & 0xFFu;
-      const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int vi = gt + i * kRowThreads;
+      const int k0 = vi << 3;
+      const uint32_t mb = vi < nvec ? (s_mask[k0 >> 5] >> (k0 & 31)) & 0xFFu : 0u;
+      const __half2 *h = reinterpret_cast<const __half2 *>(&v[i]);
       uint32_t det = 0;
 #pragma unroll
       for (int e2 = 0; e2 < 4; ++e2) {
@@ -95,41 +172,45 @@ __global__ void __launch_bounds__(kQThreads) quantize_act_kernel(
         const float a0 = fabsf(f.x), a1 = fabsf(f.y);
         if ((mb >> (2 * e2)) & 1u) aI = fmaxf(aI, a0); else aN = fmaxf(aN, a0);
         if ((mb >> (2 * e2 + 1)) & 1u) aI = fmaxf(aI, a1); else aN = fmaxf(aN, a1);
-        det |= (a0 > T ? 1u : 0u) << (2 * e2);
-        det |= (a1 > T ? 1u : 0u) << (2 * e2 + 1);
+        det |= (a0 > a.T ? 1u : 0u) << (2 * e2);
+        det |= (a1 > a.T ? 1u : 0u) << (2 * e2 + 1);
       }
       if (det) atomicOr(&s_det[k0 >> 5], det << (k0 & 31));
     }
     aI = warp_max(aI);
     aN = warp_max(aN);
     if (lane == 0) {
-      s_red[0][warp] = aI;
-      s_red[1][warp] = aN;
+      s_red[g][0][gw] = aI;
+      s_red[g][1][gw] = aN;
     }
-    __syncthreads();
-    float rI = s_red[0][0], rN = s_red[1][0];
+    named_barrier(1 + g, kRowThreads);
+    float rI = s_red[g][0][0], rN = s_red[g][1][0];
 #pragma unroll
-    for (int w = 1; w < kQWarps; ++w) {
-      rI = fmaxf(rI, s_red[0][w]);
-      rN = fmaxf(rN, s_red[1][w]);
+    for (int w = 1; w < kRowWarps; ++w) {
+      rI = fmaxf(rI, s_red[g][0][w]);
+      rN = fmaxf(rN, s_red[g][1][w]);
     }
-    __syncthreads();  // s_red is rewritten by the next row
+    named_barrier(1 + g, kRowThreads);  // s_red is rewritten by the group's next token
 
     const float amax = fmaxf(rI, rN);
-    const bool mixed = K_out > 0 && amax > T;
-    const float a = mixed ? rN : amax;
-    const float inv = a > 0.f ? __fdiv_rn(127.f, a) : 0.f;
-    if (tid == 0) {
-      s_x[m] = __fdiv_rn(a, 127.f);
+    const bool mixed = a.K_out > 0 && amax > a.T;
+    const float am = mixed ? rN : amax;
+    const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
+    if (gt == 0) {
+      a.s_x[m] = __fdiv_rn(am, 127.f);
       mixed_rows += mixed ? 1 : 0;
     }
 
-    uint2 *qr = reinterpret_cast<uint2 *>(Xq + static_cast<size_t>(m) * K);
-    for (int v = tid; v < nvec; v += kQThreads) {
-      const uint4 raw = __ldg(xr + v);
-      const int k0 = v << 3;
-      const uint32_t mb = mixed ? (s_mask[k0 >> 5] >> (k0 & 31)) & 0xFFu : 0u;
-      const __half2 *h = reinterpret_cast<const __half2 *>(&raw);
+    uint2 *qr = reinterpret_cast<uint2 *>(a.Xq + static_cast<size_t>(m) * a.K);
+    __half *orow = a.X_out + static_cast<size_t>(m) * a.K_out_pad;
+#pragma unroll
+    for (int i = 0; i < VPT; ++i) {
+      const int vi = gt + i * kRowThreads;
+      if (vi >= nvec) continue;
+      const int k0 = vi << 3;
+      const uint32_t word = s_mask[k0 >> 5];
+      const uint32_t mb = mixed ? (word >> (k0 & 31)) & 0xFFu : 0u;
+      const __half2 *h = reinterpret_cast<const __half2 *>(&v[i]);
       uint32_t lo = 0, hi = 0;
 #pragma unroll
       for (int e2 = 0; e2 < 4; ++e2) {
@@ -140,33 +221,98 @@ __global__ void __launch_bounds__(kQThreads) quantize_act_kernel(
         if (e2 < 2) lo |= pair << (16 * e2);
         else hi |= pair << (16 * (e2 - 2));
       }
-      qr[v] = make_uint2(lo, hi);
-    }
-    if (K_out_pad > 0) {
-      const __half *xh = X + static_cast<size_t>(m) * ldx;
-      __half *orow = X_out + static_cast<size_t>(m) * K_out_pad;
-      for (int j = tid; j < K_out_pad; j += kQThreads) {
-        __half v = __ushort_as_half(0);
-        if (mixed && j < K_out) {
-          const int c = s_idx[j];
-          if (c >= 0) v = xh[c];
+      qr[vi] = make_uint2(lo, hi);
+      if (mb) {  // outlier channels of a mixed token -> their X_out columns
+        const int base = static_cast<int>(s_rank[k0 >> 5]) +
+                         __popc(word & ((1u << (k0 & 31)) - 1u));
+        const unsigned short *hs = reinterpret_cast<const unsigned short *>(&v[i]);
+        int j = base;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if ((mb >> e) & 1u) {
+            orow[j] = __ushort_as_half(hs[e]);
+            ++j;
+          }
         }
-        orow[j] = v;
       }
+    }
+    // every other X_out column of this token is zero
+    for (int j = gt; j < a.K_out_pad; j += kRowThreads)
+      if (!mixed || j >= a.K_out) orow[j] = __ushort_as_half(0);
+    if (kPrefetch) {
+#pragma unroll
+      for (int i = 0; i < kVn; ++i) v[i] = vn[i];
+    } else {
+      load_row(m + row_stride, v, VPT);
     }
   }
 
-  // Publish this CTA's share of the matrix-wide outputs.
+  // ------------------------------------------- matrix-wide bitmap and flags
+  if (lane == 0) s_cnt[warp] = 0;
+  __syncwarp();
+  if ((tid % kRowThreads) == 0) s_cnt[warp] = mixed_rows;
   __syncthreads();
-  for (int w = tid; w < words; w += kQThreads) {
-    const uint32_t d = s_det[w];
-    if (d) atomicOr(&bitmap[w], d);
+  if (tid == 0) {
+    int t = 0;
+    for (int w = 0; w < G * kRowWarps; ++w) t += s_cnt[w];
+    s_part[1] = t;  // mixed tokens seen by this CTA
   }
-  if (tid == 0 && mixed_rows) atomicAdd(reinterpret_cast<int *>(&flags[0]), mixed_rows);
+  __syncthreads();
+
+  if (a.cluster_mode) {
+    const uint32_t rank = cluster_ctarank();
+    const int C = gridDim.x;
+    cluster_sync_all();  // every CTA's detection words are final
+    int outside = 0;
+    for (int w = static_cast<int>(rank) * blockDim.x + tid; w < words; w += C * blockDim.x) {
+      const uint32_t addr = smem_u32(&s_det[w]);
+      uint32_t part[kMaxClusterCtas];
+#pragma unroll
+      for (int q = 0; q < kMaxClusterCtas; ++q)  // all peers' loads in flight at once
+        part[q] = q < C ? ld_dsmem_u32(mapa_shared(addr, static_cast<uint32_t>(q))) : 0u;
+      uint32_t bits = 0;
+#pragma unroll
+      for (int q = 0; q < kMaxClusterCtas; ++q) bits |= part[q];
+      a.bitmap[w] = bits;
+      outside += __popc(bits & ~s_mask[w]);
+    }
+    outside = warp_sum(outside);
+    if (lane == 0) s_cnt[warp] = outside;
+    __syncthreads();
+    if (tid == 0) {
+      int t = 0;
+      for (int w = 0; w < G * kRowWarps; ++w) t += s_cnt[w];
+      s_part[0] = t;
+    }
+    cluster_sync_all();  // partial counts visible cluster-wide
+    if (rank == 0 && warp == 0) {  // lane q reads CTA q's counts
+      int outs = 0, mixed = 0;
+      if (lane < C) {
+        outs = static_cast<int>(ld_dsmem_u32(mapa_shared(smem_u32(&s_part[0]), lane)));
+        mixed = static_cast<int>(ld_dsmem_u32(mapa_shared(smem_u32(&s_part[1]), lane)));
+      }
+      outs = warp_sum(outs);
+      mixed = warp_sum(mixed);
+      if (lane == 0) {
+        a.flags[0] = mixed;
+        a.flags[1] = outs;
+        a.flags[2] = 0;
+        a.flags[3] = 0;
+      }
+    }
+    cluster_sync_all();  // no CTA leaves while its shared memory is still read
+    return;
+  }
+
+  for (int w = tid; w < words; w += blockDim.x) {
+    const uint32_t d = s_det[w];
+    if (d) atomicOr(&a.bitmap[w], d);
+  }
+  if (tid == 0 && s_part[1]) atomicAdd(reinterpret_cast<int *>(&a.flags[0]), s_part[1]);
   __threadfence();
   __syncthreads();
   if (tid == 0) {
-    const int prev = atomicAdd(reinterpret_cast<int *>(&flags[2]), 1);
+    const int prev = atomicAdd(reinterpret_cast<int *>(&a.flags[2]), 1);
     s_last = prev == static_cast<int>(gridDim.x) - 1;
   }
   __syncthreads();
@@ -174,41 +320,106 @@ __global__ void __launch_bounds__(kQThreads) quantize_act_kernel(
   // Last CTA: every CTA's bitmap bits are in; count detections outside idx.
   __threadfence();
   int cnt = 0;
-  for (int w = tid; w < words; w += kQThreads) cnt += __popc(__ldcg(&bitmap[w]) & ~s_mask[w]);
+  for (int w = tid; w < words; w += blockDim.x) cnt += __popc(__ldcg(&a.bitmap[w]) & ~s_mask[w]);
   cnt = warp_sum(cnt);
   if (lane == 0) s_cnt[warp] = cnt;
   __syncthreads();
   if (tid == 0) {
     int total = 0;
-    for (int w = 0; w < kQWarps; ++w) total += s_cnt[w];
-    flags[1] = total;
-    flags[2] = 0;
+    for (int w = 0; w < G * kRowWarps; ++w) total += s_cnt[w];
+    a.flags[1] = total;
+    a.flags[2] = 0;
   }
 }
 
+template <int VPT, int G>
+cudaError_t launch_variant(const QArgs &a, int grid, int cluster, cudaStream_t stream) {
+  auto kernel = quantize_act_kernel<VPT, G>;
+  const size_t smem = sizeof(uint32_t) * 3 * (a.K / 32);
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem < 48 * 1024 ? 48 * 1024 : smem));
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid, 1, 1);
+  cfg.blockDim = dim3(kRowThreads * G, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kernel, a);
+}
+
 }  // namespace
+
+int quantize_max_k() { return 16 * kRowThreads * 8; }
 
 cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx,
                                 int K_out, float threshold, int8_t *Xq, float *s_x, void *X_out,
                                 uint32_t *bitmap, int32_t *flags, int32_t *status,
                                 cudaStream_t stream, int num_sms) {
-  const int words = K / 32;
-  reset_detect_kernel<<<1, 256, 0, stream>>>(bitmap, words, flags);
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess || M == 0) return e;
-  const size_t smem = sizeof(uint32_t) * 2 * words + sizeof(int32_t) * K_out;
-  static bool configured = false;
-  if (!configured) {
-    e = cudaFuncSetAttribute(quantize_act_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             200 * 1024);
-    if (e != cudaSuccess) return e;
-    configured = true;
+  QArgs a{};
+  a.X = static_cast<const __half *>(X);
+  a.M = M;
+  a.K = K;
+  a.ldx = ldx;
+  a.idx = idx;
+  a.K_out = K_out;
+  a.K_out_pad = k_out_pad(K_out);
+  a.T = threshold;
+  a.Xq = Xq;
+  a.s_x = s_x;
+  a.X_out = static_cast<__half *>(X_out);
+  a.bitmap = bitmap;
+  a.flags = flags;
+  a.status = status;
+  const int vpt_need = (K / 8 + kRowThreads - 1) / kRowThreads;
+  const int vpt = vpt_need <= 1 ? 1 : vpt_need <= 2 ? 2 : vpt_need <= 4 ? 4 : vpt_need <= 8 ? 8 : 16;
+  // One cluster of up to 8 CTAs when that covers every token with at most 4
+  // tokens per group; G = 2 groups per CTA (1 when a row needs many
+  // registers), small enough to share an SM with a GEMM CTA.
+  const int G = vpt <= 4 ? 2 : 1;
+  const int ctas_for_m = (M + G - 1) / G;
+  if (M > 0 && ctas_for_m <= 4 * kMaxClusterCtas) {
+    const int grid = ctas_for_m < kMaxClusterCtas ? ctas_for_m : kMaxClusterCtas;
+    a.cluster_mode = 1;
+    switch (vpt) {
+      case 1: return launch_variant<1, 2>(a, grid, grid, stream);
+      case 2: return launch_variant<2, 2>(a, grid, grid, stream);
+      case 4: return launch_variant<4, 2>(a, grid, grid, stream);
+      case 8: return launch_variant<8, 1>(a, grid, grid, stream);
+      default: return launch_variant<16, 1>(a, grid, grid, stream);
+    }
   }
+  // Reset pass (waits for the preceding grid itself), then the main pass.
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, reset_detect_kernel, bitmap, K / 32, flags);
+    if (e != cudaSuccess || M == 0) return e;
+  }
+  a.cluster_mode = 0;
   const int grid = M < num_sms * 8 ? M : num_sms * 8;
-  quantize_act_kernel<<<grid, kQThreads, smem, stream>>>(
-      static_cast<const __half *>(X), M, K, ldx, idx, K_out, k_out_pad(K_out), threshold, Xq,
-      s_x, static_cast<__half *>(X_out), bitmap, flags, status);
-  return cudaGetLastError();
+  switch (vpt) {
+    case 1: return launch_variant<1, 1>(a, grid, 1, stream);
+    case 2: return launch_variant<2, 1>(a, grid, 1, stream);
+    case 4: return launch_variant<4, 1>(a, grid, 1, stream);
+    case 8: return launch_variant<8, 1>(a, grid, 1, stream);
+    default: return launch_variant<16, 1>(a, grid, 1, stream);
+  }
 }
 
 }  // namespace mixq

@@ -72,8 +72,15 @@ class Gpu:
                           else np.zeros((W.shape[0], 0), np.float16)),
                    status=int(status.item()), packed=w)
         if mode == "w8":
-            out["Wq"] = w.Wq.cpu().numpy()
+            out["Wq"] = self.unpack_w8(w)
         return out
+
+    def unpack_w8(self, w):
+        torch, mq = self.torch, self.mq
+        out = torch.empty((w.N, w.K), dtype=torch.int8, device="cuda")
+        mq.mixq_debug_unpack_w8(w.N, w.K, w.Wq, out)
+        torch.cuda.synchronize()
+        return out.cpu().numpy()
 
     def unpack_w4(self, w):
         torch, mq = self.torch, self.mq
