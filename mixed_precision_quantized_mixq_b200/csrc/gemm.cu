@@ -208,18 +208,6 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
         mbar_arrive_expect_tx(&full[j], a_bytes + b_bytes);
         issue_b(j, j, pol_b);
       }
-      // When this CTA is the only reader of its weights (one row tile of
-      // tokens), pull the rest of its weight slice into L2 now as well: the
-      // HBM stream then runs ahead of the pipeline, across the wait for the
-      // preceding kernel and across this CTA's own stage recycling.
-      if (p.b_streamed) {
-        for (int j = pre; j < n_i8; ++j) {
-          for (int h = 0; h < n_sub; ++h) {
-            prefetch_l2(w_src(kb_begin + j, h), C::kSubRows * C::kRowW);
-            if (W4) prefetch_l2(g_src(kb_begin + j, h), C::kSubRows * 4);
-          }
-        }
-      }
     }
     tma_prefetch_desc(&tm_a);
     if (!RAW && p.K_out_pad > 0 && rank == 0) {
@@ -786,16 +774,15 @@ GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimi
     // Decode-sized M is latency bound: a CTA streams one 16 KB weight stage
     // per ~0.4 us whatever the tile width (measured), so what matters is how
     // many CTAs stream at once.  128-wide tiles, K split into the smallest
-    // cluster that brings the CTA count to about one per SM (never past
-    // 1.25 per SM, never past one wave of clusters).
+    // cluster that brings the CTA count to about one per SM, never past
+    // 1.25 per SM (a small-M CTA leaves room for a second one on its SM).
+    (void)limits;
     const int KB = K / kBlockK;
     const int n_tiles = N / 128;
     int best_s = 1;
     for (int s = 1; s <= 8 && s <= KB; ++s) {
       const int ctas = n_tiles * s;
-      const int clusters_per_wave =
-          limits ? limits->max_active[1][0][s] : estimate_max_active_clusters(num_sms, 2, s);
-      if (ctas > num_sms + num_sms / 4 || n_tiles > clusters_per_wave) break;
+      if (ctas > num_sms + num_sms / 4) break;
       best_s = s;
       if (ctas * 5 >= num_sms * 4) break;
     }
