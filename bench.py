@@ -184,6 +184,29 @@ class ClockSampler:
                 "samples": len(inside)}
 
 
+# ------------------------------------------------------- multi-rank helpers
+def rank_activations(case, rank: int):
+    """Activations of one case for one rank: rank 0 uses the workload's own
+    seeded tensor, rank r > 0 an independent draw (seed offset 1000 r) of the
+    same distribution -- each rank processes its own batch (weak scaling)."""
+    idx = case.channels()
+    seed = synth.SEED_X + 1000 * rank
+    if case.scaled and case.k_out:
+        f = case.factor if case.factor is not None else synth.channel_factors(case.k_out)
+        return synth.activations(case.M, case.K, idx, f, seed=seed), idx
+    return synth.activations(case.M, case.K, seed=seed), idx
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Largest value across ranks (a no-op for one rank)."""
+    if world <= 1:
+        return value
+    import torch
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
 # ----------------------------------------------------------------- GPU arm
 def run_gpu(args, rank, world):
     import torch
@@ -199,11 +222,7 @@ def run_gpu(args, rank, world):
     weights_host = {}
     layers = []
     for ci, (case, modes) in enumerate(cases):
-        X, _, idx = case.make()
-        if rank:
-            X = synth.activations(case.M, case.K, idx, synth.channel_factors(case.k_out),
-                                  seed=synth.SEED_X + 1000 * rank) if case.k_out else \
-                synth.activations(case.M, case.K, seed=synth.SEED_X + 1000 * rank)
+        X, idx = rank_activations(case, rank)
         key = (case.N, case.K)
         if key not in weights_host:
             weights_host[key] = synth.weights(case.N, case.K)
@@ -297,10 +316,7 @@ def run_gpu(args, rank, world):
     clocks = sampler.stop()
     mq.check_status(status)
 
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(total_ms, world, dev)
 
     # ---- per-kernel durations from the in-graph phase events
     kinds = {"quantize": [0.0, 0.0, 0], "gemm_w8": [0.0, 0.0, 0], "gemm_w4": [0.0, 0.0, 0]}
@@ -380,10 +396,7 @@ def run_gpu(args, rank, world):
     e2.record()
     torch.cuda.synchronize()
     e2e_ms = s2.elapsed_time(e2)
-    if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, world, dev)
     mq.check_status(status)
     e2e = {"value": round(ops_step * world / (e2e_ms / args.steps * 1e-3) / 1e12, 4),
            "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
