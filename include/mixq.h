@@ -176,8 +176,8 @@ mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
  * output tile width *bn (32, 64, 128 or 256 columns; tiles are 128 rows
  * high), the K-split factor *split (thread-block cluster size along K, 1..8)
  * and the number of CTAs *ctas.  num_sms <= 0 means "query the current
- * device" (and its cluster occupancy).  For M <= 64 and bn <= 128 the plan
- * runs the small-M variant (token-sized A slots, two CTAs per SM).
+ * device" (and its cluster occupancy).  With bn <= 128 the plan runs the
+ * variant that fits two CTAs per SM (token-sized A slots when M <= 64).
  */
 mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, int *split,
                            int *ctas);

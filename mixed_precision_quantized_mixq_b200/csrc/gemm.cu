@@ -128,6 +128,7 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
     mixq_gemm_kernel(const __grid_constant__ CUtensorMap tm_a,   // Xq   [M][K] int8
                      const __grid_constant__ CUtensorMap tm_xo,  // X_out [M][K_out_pad] fp16
                      const __grid_constant__ CUtensorMap tm_wo,  // W_out [N][K_out_pad] fp16
+                     const __grid_constant__ CUtensorMap tm_y,   // Y [M][ldy] fp16 (store)
                      const KParams p) {
   using C = Cfg<BN, W4, SM>;
   extern __shared__ uint8_t smem_raw[];
@@ -369,7 +370,63 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
   const bool failed = *s_err != 0;
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
 
-  if (S == 1) {
+  if (S == 1 && !RAW && BN >= 64) {
+    // Stage the fp16 tile in shared memory in the 128-byte swizzled layout of
+    // a TMA store (64-column sub-tiles of a_rows rows; a thread's 16-byte
+    // pieces of one row land on 8 different bank groups), then one thread
+    // writes it out with coalesced bulk tensor stores.
+    uint8_t *stage_y = ring;  // the ring is free: every MMA has completed
+    const int box_rows = p.a_rows;
+    if (warp < 4 && !failed) {
+      const int row = warp * 32 + lane;
+      const float sx = s_sx[row];
+#pragma unroll 1
+      for (int c = 0; c < BN / 32; ++c) {
+        if (n0 + c * 32 >= p.N) break;
+        uint32_t acc[32], o[32];
+        tmem_ld32(tmem_base + lane_base + c * 32, acc);
+        if (do_out) tmem_ld32(tmem_base + lane_base + BN + c * 32, o);
+        tmem_ld_wait();
+        if (row < box_rows) {
+          const float4 *sw4 = reinterpret_cast<const float4 *>(s_sw + c * 32);
+          uint32_t h[16];
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 w = sw4[i];
+            const float wv[4] = {w.x, w.y, w.z, w.w};
+            float y[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int q = 4 * i + e;
+              float v = __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(acc[q])), sx),
+                                  wv[e]);
+              if (do_out) v = __fadd_rn(v, __uint_as_float(o[q]));
+              y[e] = v;
+            }
+            const __half2 h0 = __floats2half2_rn(y[0], y[1]);
+            const __half2 h1 = __floats2half2_rn(y[2], y[3]);
+            h[2 * i] = *reinterpret_cast<const uint32_t *>(&h0);
+            h[2 * i + 1] = *reinterpret_cast<const uint32_t *>(&h1);
+          }
+          uint8_t *rowp = stage_y + (c >> 1) * box_rows * 128 + row * 128;
+          const int j0 = (c & 1) * 4;
+#pragma unroll
+          for (int q = 0; q < 4; ++q)
+            *reinterpret_cast<uint4 *>(rowp + (((j0 + q) ^ (row & 7)) << 4)) =
+                make_uint4(h[4 * q], h[4 * q + 1], h[4 * q + 2], h[4 * q + 3]);
+        }
+      }
+      fence_proxy_async_smem();
+    }
+    if (warp < 4) named_barrier(1, 128);
+    if (threadIdx.x == 0 && !failed) {
+      const int cols = min(BN, p.N - n0);
+      for (int t = 0; t < cols / 64; ++t)
+        tma_store_2d(&tm_y, stage_y + t * box_rows * 128, n0 + t * 64, m0);
+      bulk_commit_group();
+      bulk_wait_all();
+    }
+  } else if (S == 1) {
     if (warp < 4 && !failed) {
       const int row = warp * 32 + lane;
       const int m = m0 + row;
@@ -603,7 +660,7 @@ Geometry geometry(int M, int split) {
     g.stages = C::kStages;
     g.a_stride = kTileM * kBlockK;
   } else {
-    const int a_rows = M >= 64 ? 64 : (M + 7) / 8 * 8;
+    const int a_rows = M >= kTileM ? kTileM : (M + 7) / 8 * 8;  // = the TMA box rows
     g.a_stride = a_rows * kBlockK;
     const int budget = 233472 / 2 - 1024 - C::kExtra - 1024;  // half an SM, minus reserve
     g.stages = budget / (g.a_stride + C::kBStage);
@@ -640,9 +697,10 @@ cudaError_t launch_variant(const GemmArgs &a, const GemmPlan &plan, cudaStream_t
 
   const int kp = k_out_pad(a.K_out);
   const int a_rows = a.M >= kTileM ? kTileM : (a.M + 7) / 8 * 8;
-  alignas(64) CUtensorMap tm_a, tm_xo, tm_wo;
+  alignas(64) CUtensorMap tm_a, tm_xo, tm_wo, tm_y;
   memset(&tm_xo, 0, sizeof tm_xo);
   memset(&tm_wo, 0, sizeof tm_wo);
+  memset(&tm_y, 0, sizeof tm_y);
   bool ok = make_map(&tm_a, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, a.Xq, a.K, a.M, a.K, kBlockK,
                      a_rows, CU_TENSOR_MAP_SWIZZLE_128B);
   if (a.epi != Epi::kRawI32 && kp > 0) {
@@ -653,6 +711,10 @@ cudaError_t launch_variant(const GemmArgs &a, const GemmPlan &plan, cudaStream_t
                         static_cast<uint64_t>(kp) * 2, kOutBlockK, BN,
                         CU_TENSOR_MAP_SWIZZLE_128B);
   }
+  if (a.epi != Epi::kRawI32 && BN >= 64)
+    ok = ok && make_map(&tm_y, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, a.Y, a.N, a.M,
+                        static_cast<uint64_t>(a.ldy) * 2, 64, a_rows,
+                        CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) {
     *why = "cuTensorMapEncodeTiled failed (or the driver entry point is unavailable)";
     return cudaErrorInvalidValue;
@@ -697,7 +759,7 @@ cudaError_t launch_variant(const GemmArgs &a, const GemmPlan &plan, cudaStream_t
   attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
-  return cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_xo, tm_wo, kp_);
+  return cudaLaunchKernelEx(&cfg, kernel, tm_a, tm_xo, tm_wo, tm_y, kp_);
 }
 
 template <int BN, bool W4, bool SM>
@@ -798,9 +860,23 @@ GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimi
   // Memory: the bytes that must come from HBM at least once (weights,
   // activations, output) at the HBM rate.  Cost = max(compute, memory); ties
   // keep fewer CTAs.
+  const int m_tiles = (M + kTileM - 1) / kTileM;
+  {
+    // Prefill-sized M.  W8: two 128 x 128 CTAs per SM (about 100 KB each), so
+    // one CTA's epilogue overlaps the other's mainloop and the grid packs
+    // into waves twice as finely (measured better than one 128 x 256 CTA per
+    // SM on every workload shape).  W4: its expansion needs the deeper
+    // one-CTA-per-SM pipeline, unless that grid wastes more than 15% of its
+    // last wave.
+    const int n128 = (N + 127) / 128;
+    if (mode != 1) return GemmPlan{128, 1, m_tiles * n128, 1};
+    const long long ctas256 = static_cast<long long>(m_tiles) * ((N + 255) / 256);
+    const double waves = static_cast<double>(ctas256) / num_sms;
+    const double tail_eff = waves / static_cast<double>((ctas256 + num_sms - 1) / num_sms);
+    if (tail_eff < 0.85) return GemmPlan{128, 1, m_tiles * n128, 1};
+  }
   GemmPlan best{256, 1, 0, 0};
   double best_cost = 1e300;
-  const int m_tiles = (M + kTileM - 1) / kTileM;
   const int KB = K / kBlockK;
   const double w_bytes = (mode == 1 ? 0.5 + 4.0 / kGroup : 1.0) * static_cast<double>(N) * K;
   const double unique_bytes = w_bytes + static_cast<double>(M) * K + 2.0 * M * N;
