@@ -284,7 +284,9 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms, mixq::device_cluster_limits(mode));
   if (bn) plan.bn = bn;
   if (split) plan.split = split;
-  if (bn || split) plan.small_m = plan.bn <= 128 ? 1 : 0;
+  // two-CTA-per-SM variant for bn <= 128, except a K split with more rows
+  // than its reduction buffers hold (64)
+  if (bn || split) plan.small_m = (plan.bn <= 128 && (M <= 64 || plan.split == 1)) ? 1 : 0;
   mixq::GemmArgs a{};
   a.mode = mode;
   a.M = M;

@@ -688,6 +688,11 @@ cudaError_t launch_variant(const GemmArgs &a, const GemmPlan &plan, cudaStream_t
   auto kernel = mixq_gemm_kernel<BN, W4, SM, RAW>;
   cudaError_t e = ensure_smem(kernel, max_smem<BN, W4, SM>(), smem_done);
   if (e != cudaSuccess) return e;
+  if (plan.split > 1 && a.M > C::kRedRows && (a.M + kTileM - 1) / kTileM * kTileM > C::kRedRows &&
+      C::kRedRows < kTileM) {
+    *why = "a K split of this variant reduces at most 64 rows per tile";
+    return cudaErrorInvalidValue;
+  }
   const Geometry geo = geometry<BN, W4, SM>(a.M, plan.split);
   if (geo.smem > max_smem<BN, W4, SM>() || geo.stages < 2 ||
       (plan.split > 1 && C::ring_bytes(geo.stages, geo.a_stride) < C::kRedBytes)) {
