@@ -231,12 +231,27 @@ def run_gpu(args, rank, world):
         packed = {m: mq.prepack(Wd, idxd, mq.MIXQ_W8 if m == "w8" else mq.MIXQ_W4G128)
                   for m in modes}
         del Wd
-        Xd = torch.from_numpy(X).to(dev)
-        q = mq.quantize_act(Xd, idxd, T)
-        Ys = {m: torch.empty((case.M, case.N), dtype=torch.float16, device=dev) for m in modes}
-        layers.append(dict(case=case, modes=modes, X=Xd, idx=idxd, q=q, packed=packed, Y=Ys))
-    torch.cuda.synchronize()
+        layers.append(dict(case=case, modes=modes, Xh=X, idx=idxd, packed=packed))
     weights_host.clear()
+    # All activations of a step live in one device buffer and all outputs in
+    # another (per-case views), so the end-to-end leg moves each with a single
+    # host<->device copy.
+    x_sizes = [L["case"].M * L["case"].K for L in layers]
+    y_sizes = [L["case"].M * L["case"].N * len(L["modes"]) for L in layers]
+    X_all = torch.empty(sum(x_sizes), dtype=torch.float16, device=dev)
+    Y_all = torch.empty(sum(y_sizes), dtype=torch.float16, device=dev)
+    xo = yo = 0
+    for L, xs, ys in zip(layers, x_sizes, y_sizes):
+        c = L["case"]
+        L["X"] = X_all[xo:xo + xs].view(c.M, c.K)
+        L["X"].copy_(torch.from_numpy(L.pop("Xh")))
+        L["Y"] = {}
+        for mi, m in enumerate(L["modes"]):
+            L["Y"][m] = Y_all[yo + mi * c.M * c.N: yo + (mi + 1) * c.M * c.N].view(c.M, c.N)
+        L["q"] = mq.quantize_act(L["X"], L["idx"], T)
+        xo += xs
+        yo += ys
+    torch.cuda.synchronize()
 
     status = torch.zeros(1, dtype=torch.int32, device=dev)
 
@@ -367,19 +382,15 @@ def run_gpu(args, rank, world):
                                    for k, v in kinds.items()}})
 
     # ---- end to end: host X in pinned memory -> device -> layer -> Y back to pinned host
-    host_X = [L["X"].cpu().pin_memory() for L in layers]
-    host_Y = [{m: torch.empty(L["Y"][m].shape, dtype=torch.float16).pin_memory() for m in L["modes"]}
-              for L in layers]
-    h2d = sum(x.numel() * 2 for x in host_X)
-    d2h = sum(y.numel() * 2 for d in host_Y for y in d.values())
+    host_X = X_all.cpu().pin_memory()
+    host_Y = torch.empty(Y_all.shape, dtype=torch.float16).pin_memory()
+    h2d = host_X.numel() * 2
+    d2h = host_Y.numel() * 2
 
     def e2e_step():
-        for li, L in enumerate(layers):
-            L["X"].copy_(host_X[li], non_blocking=True)
-            mq.quantize_act(L["X"], L["idx"], T, out=L["q"], status=status)
-            for m in L["modes"]:
-                mq.gemm(L["q"], L["packed"][m], Y=L["Y"][m], status=status)
-                host_Y[li][m].copy_(L["Y"][m], non_blocking=True)
+        X_all.copy_(host_X, non_blocking=True)
+        step()
+        host_Y.copy_(Y_all, non_blocking=True)
 
     ge = torch.cuda.CUDAGraph()
     with torch.cuda.graph(ge, stream=side):
@@ -401,7 +412,8 @@ def run_gpu(args, rank, world):
     e2e = {"value": round(ops_step * world / (e2e_ms / args.steps * 1e-3) / 1e12, 4),
            "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": round(e2e_ms / args.steps, 5),
-           "how": "pinned host X -> device, quantize + both GEMMs, Y -> pinned host; CUDA graph"}
+           "how": "one pinned-host -> device copy of every case's X, quantize + both GEMMs, one "
+                  "device -> pinned-host copy of every Y; CUDA graph"}
 
     # quantize is one kernel for decode-sized M (one cluster), else reset + main pass
     launches_per_step = sum((1 if L["case"].M <= (64 if L["case"].K <= 8192 else 32) else 2)

@@ -86,6 +86,7 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
   uint32_t *s_rank = qsm + 2 * words;   // outlier channels in words before w
   __shared__ float s_red[G][2][kRowWarps];
   __shared__ int s_bad, s_last, s_part[2], s_cnt[G * kRowWarps];
+  __shared__ uint32_t s_mixed_total;  // cluster mode: rank 0 accumulates every CTA's count
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = tid / kRowThreads, gt = tid % kRowThreads, gw = gt >> 5;
@@ -108,8 +109,14 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
     s_mask[w] = 0u;
     s_det[w] = 0u;
   }
-  if (tid == 0) s_bad = 0;
+  if (tid == 0) {
+    s_bad = 0;
+    s_mixed_total = 0u;
+  }
   __syncthreads();
+  // cluster mode: signal that this CTA's accumulators are initialised; the
+  // matching wait comes before any CTA adds into rank 0's
+  if (a.cluster_mode) cluster_arrive_relaxed();
   for (int j = tid; j < a.K_out; j += blockDim.x) {
     const int c = a.idx[j];
     const bool ok = c >= 0 && c < a.K && (j == 0 || a.idx[j - 1] < c);
@@ -260,19 +267,24 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
   __syncthreads();
 
   if (a.cluster_mode) {
+    // Every CTA ORs its detection words and adds its mixed-token count into
+    // CTA rank 0's shared memory; after one cluster barrier rank 0 owns the
+    // matrix-wide result and no CTA reads another's memory again.
     const uint32_t rank = cluster_ctarank();
-    const int C = gridDim.x;
-    cluster_sync_all();  // every CTA's detection words are final
+    cluster_wait();  // rank 0's accumulators are initialised
+    if (rank != 0) {
+      for (int w = tid; w < words; w += blockDim.x) {
+        const uint32_t d = s_det[w];
+        if (d) red_or_dsmem(mapa_shared(smem_u32(&s_det[w]), 0u), d);
+      }
+    }
+    if (tid == 0)
+      red_add_dsmem(mapa_shared(smem_u32(&s_mixed_total), 0u), static_cast<uint32_t>(s_part[1]));
+    cluster_sync_all();  // every CTA's contributions have landed in rank 0
+    if (rank != 0) return;
     int outside = 0;
-    for (int w = static_cast<int>(rank) * blockDim.x + tid; w < words; w += C * blockDim.x) {
-      const uint32_t addr = smem_u32(&s_det[w]);
-      uint32_t part[kMaxClusterCtas];
-#pragma unroll
-      for (int q = 0; q < kMaxClusterCtas; ++q)  // all peers' loads in flight at once
-        part[q] = q < C ? ld_dsmem_u32(mapa_shared(addr, static_cast<uint32_t>(q))) : 0u;
-      uint32_t bits = 0;
-#pragma unroll
-      for (int q = 0; q < kMaxClusterCtas; ++q) bits |= part[q];
+    for (int w = tid; w < words; w += blockDim.x) {
+      const uint32_t bits = s_det[w];
       a.bitmap[w] = bits;
       outside += __popc(bits & ~s_mask[w]);
     }
@@ -282,25 +294,11 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
     if (tid == 0) {
       int t = 0;
       for (int w = 0; w < G * kRowWarps; ++w) t += s_cnt[w];
-      s_part[0] = t;
+      a.flags[0] = static_cast<int32_t>(s_mixed_total);
+      a.flags[1] = t;
+      a.flags[2] = 0;
+      a.flags[3] = 0;
     }
-    cluster_sync_all();  // partial counts visible cluster-wide
-    if (rank == 0 && warp == 0) {  // lane q reads CTA q's counts
-      int outs = 0, mixed = 0;
-      if (lane < C) {
-        outs = static_cast<int>(ld_dsmem_u32(mapa_shared(smem_u32(&s_part[0]), lane)));
-        mixed = static_cast<int>(ld_dsmem_u32(mapa_shared(smem_u32(&s_part[1]), lane)));
-      }
-      outs = warp_sum(outs);
-      mixed = warp_sum(mixed);
-      if (lane == 0) {
-        a.flags[0] = mixed;
-        a.flags[1] = outs;
-        a.flags[2] = 0;
-        a.flags[3] = 0;
-      }
-    }
-    cluster_sync_all();  // no CTA leaves while its shared memory is still read
     return;
   }
 
