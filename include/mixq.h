@@ -162,7 +162,9 @@ mixq_status mixq_gemm_w8a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
  * Same layer with 4-bit group-wise weights (QServe 渐进量化 / 寄存器压力和并行性,
  * MixLLM two-stage dequantization): inside the mainloop every 4-bit code is
  * expanded back to the INT8 weight (q - z2)*s2, four codes per 32-bit
- * register operation, and multiplied on INT8 tensor cores.
+ * register operation, and multiplied on INT8 tensor cores.  The expanded
+ * weights go from registers into tensor memory and are the MMA's A operand
+ * (tokens are B), so each CTA owns 128 output channels x up to 128 tokens.
  *   Wq4/grp/s_w/W_out from mixq_prepack_weights(MIXQ_W4G128); the rest as
  *   mixq_gemm_w8a8o16.
  */
@@ -173,20 +175,26 @@ mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
 
 /*
  * The launch plan the gemm calls use for a shape (host only, no GPU needed):
- * output tile width *bn (32, 64, 128 or 256 columns; tiles are 128 rows
- * high), the K-split factor *split (thread-block cluster size along K, 1..8)
- * and the number of CTAs *ctas.  num_sms <= 0 means "query the current
- * device" (and its cluster occupancy).  With bn <= 128 the plan runs the
- * variant that fits two CTAs per SM (token-sized A slots when M <= 64).
+ * output tile width *bn in output channels (MIXQ_W8: 32, 64, 128 or 256, tiles
+ * 128 tokens high; MIXQ_W4G128: always 128, tiles of up to 128 tokens, all
+ * tokens when M <= 64), the K-split factor *split (thread-block cluster size
+ * along K, 1..8) and the number of CTAs *ctas.  num_sms <= 0 means "query the
+ * current device" (and, for MIXQ_W8, its cluster occupancy).  MIXQ_W8 with
+ * bn <= 128 runs the variant that fits two CTAs per SM (token-sized A slots
+ * when M <= 64).
  */
 mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, int *split,
                            int *ctas);
 
 /*
  * Test-only: the gemm mainloop alone, raw INT32 accumulators out
- * (acc int32 [M][ldacc]).  mode MIXQ_W8 uses Wq; MIXQ_W4G128 uses Wq4 + grp.
- * bn/split override the plan when > 0 (bn 32 and 64 need M <= 64; with
- * M <= 64 and bn <= 128 the small-M variant runs).
+ * (acc int32 [M][ldacc], ldacc % 4 == 0).  mode MIXQ_W8 uses Wq; MIXQ_W4G128
+ * uses Wq4 + grp.  bn/split override the plan when > 0.  MIXQ_W8: bn 32 and
+ * 64 need M <= 64; with M <= 64 and bn <= 128 the small-M variant runs.
+ * MIXQ_W4G128: bn 128 = the tensor-memory-operand kernel's two-CTA-per-SM
+ * variant (a K split only with M <= 64, else MIXQ_ERR_UNSUPPORTED_SHAPE),
+ * 256 = its one-CTA-per-SM variant, 32/64 = the shared-memory-operand
+ * kernel with narrow tiles (M <= 64).
  */
 mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq, const void *Wq,
                                 const void *grp, int32_t *acc, int ldacc, int bn, int split,

@@ -205,8 +205,9 @@ static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const i
   a.epi = mixq::Epi::kMixed;
   a.status = status;
   a.wait_limit_ns = kDefaultWaitNs;
-  const mixq::GemmPlan plan =
-      mixq::plan_gemm(mode, M, N, K, sms, mixq::device_cluster_limits(mode));
+  // (the decode-sized W4 planner needs no occupancy table)
+  const mixq::GemmPlan plan = mixq::plan_gemm(
+      mode, M, N, K, sms, (mode == MIXQ_W8 || M > 64) ? mixq::device_cluster_limits(mode) : nullptr);
   const char *why = nullptr;
   const cudaError_t e = mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why);
   return from_cuda(e, "gemm launch", why);
@@ -273,6 +274,9 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   if (split < 0 || split > 8)
     return fail(MIXQ_ERR_INVALID_ARG, "split = %d", split);
   if (split > K / 128) return fail(MIXQ_ERR_UNSUPPORTED_SHAPE, "split %d exceeds K/128", split);
+  if (mode == MIXQ_W4G128 && bn == 128 && split > 1 && M > 64)
+    return fail(MIXQ_ERR_UNSUPPORTED_SHAPE,
+                "W4 two-CTA variant (bn = 128) splits K only for M <= 64");
   if (M == 0) return check_device(nullptr);
   if (!Xq || !Wq || !acc || (mode == MIXQ_W4G128 && !grp))
     return fail(MIXQ_ERR_INVALID_ARG, "null pointer");
@@ -281,12 +285,23 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   int sms = 0;
   s = check_device(&sms);
   if (s != MIXQ_OK) return s;
-  mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms, mixq::device_cluster_limits(mode));
-  if (bn) plan.bn = bn;
+  mixq::GemmPlan plan = mixq::plan_gemm(
+      mode, M, N, K, sms, (mode == MIXQ_W8 || M > 64) ? mixq::device_cluster_limits(mode) : nullptr);
   if (split) plan.split = split;
-  // two-CTA-per-SM variant for bn <= 128, except a K split with more rows
-  // than its reduction buffers hold (64)
-  if (bn || split) plan.small_m = (plan.bn <= 128 && (M <= 64 || plan.split == 1)) ? 1 : 0;
+  if (mode == MIXQ_W4G128 && (bn == 128 || bn == 256 || (bn == 0 && plan.ts))) {
+    // tensor-memory-operand kernel: bn = 128 the two-CTA-per-SM variant,
+    // 256 the one-CTA variant, 0 the planner's choice
+    if (bn == 128) plan.small_m = 1;
+    if (bn == 256) plan.small_m = 0;
+    plan.bn = 128;
+    plan.ts = 1;
+  } else {
+    plan.ts = 0;
+    if (bn) plan.bn = bn;
+    // two-CTA-per-SM variant for bn <= 128, except a K split with more rows
+    // than its reduction buffers hold (64)
+    if (bn || split) plan.small_m = (plan.bn <= 128 && (M <= 64 || plan.split == 1)) ? 1 : 0;
+  }
   mixq::GemmArgs a{};
   a.mode = mode;
   a.M = M;

@@ -35,6 +35,7 @@
 
 #include "internal.h"
 #include "ptx.cuh"
+#include "tma_host.h"
 
 namespace mixq {
 namespace {
@@ -591,59 +592,6 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
 }
 
 // ------------------------------------------------------------------ host side
-using EncodeTiledFn = CUresult (*)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
-                                   const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
-                                   const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
-                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-
-EncodeTiledFn encode_fn() {
-  static EncodeTiledFn fn = nullptr;
-  static std::once_flag once;
-  std::call_once(once, [] {
-    void *p = nullptr;
-    cudaDriverEntryPointQueryResult q;
-    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
-            cudaSuccess &&
-        q == cudaDriverEntryPointSuccess)
-      fn = reinterpret_cast<EncodeTiledFn>(p);
-  });
-  return fn;
-}
-
-// Row-major 2-D tensor [outer][inner] of `elem` bytes per element.
-bool make_map(CUtensorMap *map, CUtensorMapDataType dt, int elem, const void *base,
-              uint64_t inner, uint64_t outer, uint64_t row_bytes, uint32_t box_inner,
-              uint32_t box_outer, CUtensorMapSwizzle sw) {
-  EncodeTiledFn fn = encode_fn();
-  if (!fn) return false;
-  cuuint64_t dims[2] = {inner, outer};
-  cuuint64_t strides[1] = {row_bytes};
-  cuuint32_t box[2] = {box_inner, box_outer};
-  cuuint32_t estr[2] = {1, 1};
-  (void)elem;
-  return fn(map, dt, 2, const_cast<void *>(base), dims, strides, box, estr,
-            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
-}
-
-// cudaFuncSetAttribute once per (kernel, device).
-template <typename K>
-cudaError_t ensure_smem(K kernel, int bytes, std::atomic<uint64_t> &done_mask) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  const uint64_t bit = 1ull << (dev & 63);
-  if (done_mask.load(std::memory_order_acquire) & bit) return cudaSuccess;
-  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-  // all of the unified L1/shared array as shared memory, so that two small-M
-  // CTAs (about 106 KB each) fit on one SM
-  if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(kernel, cudaFuncAttributePreferredSharedMemoryCarveout,
-                             cudaSharedmemCarveoutMaxShared);
-  if (e == cudaSuccess) done_mask.fetch_or(bit, std::memory_order_acq_rel);
-  return e;
-}
-
 // Pipeline geometry of a launch: stage count, A slot size, dynamic smem.
 // Full-size variants use 128-row A slots and a fixed depth; the small-M
 // variant sizes its A slots to the token rows and takes as many stages as fit
@@ -837,6 +785,10 @@ int estimate_max_active_clusters(int num_sms, int ctas_per_sm, int split) {
 }
 
 GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimits *limits) {
+  // W4 at decode-sized M: expanded weights in tensor memory (measured 1.4x
+  // faster than the smem operand at M = 16; slower at M = 2048, where the
+  // smem x smem kernel below keeps W4)
+  if (mode == 1 && M <= 64) return plan_gemm_w4ts(M, N, K, num_sms);
   if (M <= 64) {
     // Decode-sized M is latency bound: a CTA streams one 16 KB weight stage
     // per ~0.4 us whatever the tile width (measured), so what matters is how
@@ -921,6 +873,7 @@ GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimi
 
 cudaError_t launch_gemm(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
                         const char **why) {
+  if (a.mode == 1 && plan.ts) return launch_gemm_w4ts(a, plan, stream, why);
   const bool w4 = a.mode == 1;
   const bool raw = a.epi == Epi::kRawI32;
 #define MIXQ_DISPATCH(BN_, SM_)                                                      \

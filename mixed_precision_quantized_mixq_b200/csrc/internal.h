@@ -34,10 +34,11 @@ cudaError_t launch_unpack_w4(int N, int K, const void *Wq4, const void *grp, uin
 
 // -------------------------------------------------------------------- gemm
 struct GemmPlan {
-  int bn;       // output tile width (128 or 256)
+  int bn;       // output tile width in weight rows (32..256; always 128 for W4)
   int split;    // K split = cluster size along z (1..8)
   int ctas;     // total CTAs launched
-  int small_m;  // M <= 64 kernel variant (two CTAs per SM), bn == 128 only
+  int small_m;  // two-CTA-per-SM kernel variant (half the shared memory and TMEM)
+  int ts;       // W4 through the tensor-memory-operand kernel (gemm_w4ts.cu)
 };
 
 // How many clusters of `split` CTAs run at once, per [small-M][bn == 256][split].
@@ -71,8 +72,14 @@ struct GemmArgs {
   int debug_stall;  // producer issues nothing (timeout test)
 };
 
+// W8, and W4 at prefill-sized M, run the smem x smem kernel (gemm.cu); W4 at
+// decode-sized M runs the kernel that keeps the expanded weights in tensor
+// memory (gemm_w4ts.cu, plan.ts = 1).
 cudaError_t launch_gemm(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
                         const char **why);
+GemmPlan plan_gemm_w4ts(int M, int N, int K, int num_sms);
+cudaError_t launch_gemm_w4ts(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
+                             const char **why);
 
 // Device properties cached per device.
 int device_sm_count(int dev);

@@ -280,6 +280,18 @@ __device__ __forceinline__ uint64_t sw128_kmajor_desc(uint32_t smem_addr) {
 
 // Instruction descriptors (dense, no negation, both operands K-major).
 // bits 4-5 accumulator format, 7-9 A format, 10-12 B format, 17-22 N>>3, 24-28 M>>4.
+// Same for a K-major tile with 64-byte rows in the 64-byte swizzle (8-row
+// groups 512 bytes apart).
+__device__ __forceinline__ uint64_t sw64_kmajor_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>(1u) << 16;
+  d |= static_cast<uint64_t>(512u >> 4) << 32;
+  d |= static_cast<uint64_t>(1u) << 46;
+  d |= static_cast<uint64_t>(4u) << 61;
+  return d;
+}
+
 __host__ __device__ constexpr uint32_t idesc_s8_s32(int m, int n) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);

@@ -99,3 +99,17 @@ def test_gemm_plan(lib, M, N, K):
         assert ctas >= 64
     if M >= 2048:
         assert split == 1
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 11008, 4096), (64, 4096, 11008),
+                                   (100, 4096, 4096), (512, 4096, 4096), (2048, 11008, 4096),
+                                   (512, 28672, 8192), (512, 8192, 28672)])
+def test_gemm_plan_w4(lib, M, N, K):
+    bn, split, ctas = mq.mixq_gemm_plan(mq.MIXQ_W4G128, M, N, K, 148)
+    assert 1 <= split <= 8 and split <= K // 128
+    if M <= 64:
+        # tensor-memory-operand kernel: 128 weight rows x all tokens per tile
+        assert bn == 128 and ctas == (N // 128) * split
+        assert 64 <= ctas <= 148 + 148 // 4
+    else:
+        assert bn in (128, 256) and ctas == -(-M // 128) * -(-N // bn) * split
