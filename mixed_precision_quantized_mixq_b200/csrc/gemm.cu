@@ -221,10 +221,6 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
     tmem_alloc(tmem_holder, C::kTmemCols);
     tmem_relinquish();
   }
-  if (!RAW && (warp == 2 || warp == 3)) {
-    // per-channel weight scales of the tile (read only here, never in the epilogue loop)
-    for (int i = threadIdx.x - 64; i < BN; i += 64) s_sw[i] = n0 + i < p.N ? p.s_w[n0 + i] : 0.f;
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -302,6 +298,10 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
     }
   } else if ((warp == 2 || warp == 3) && !RAW) {
     // ------------------------------------ token scales of the tile, early
+    // per-channel weight scales first (they do not depend on the preceding
+    // kernel), then the token scales; both during the mainloop, off the
+    // set-up path (a global read there delays every role by its latency)
+    for (int i = threadIdx.x - 64; i < BN; i += 64) s_sw[i] = n0 + i < p.N ? p.s_w[n0 + i] : 0.f;
     griddep_wait();
     for (int i = threadIdx.x - 64; i < kTileM; i += 64)
       s_sx[i] = m0 + i < p.M ? p.s_x[m0 + i] : 0.f;
@@ -784,28 +784,33 @@ int estimate_max_active_clusters(int num_sms, int ctas_per_sm, int split) {
   return gpcs * ((per_gpc * ctas_per_sm) / split);
 }
 
+int decode_split(int n_tiles, int KB, int num_sms) {
+  // Decode-sized M is latency bound: each CTA works through its K blocks one
+  // pipeline round trip at a time, so the time falls with the K blocks per
+  // CTA until the fixed per-CTA cost (set-up, first load, cluster reduction)
+  // dominates.  Measured on 4096/11008-wide Llama shapes (W8 and W4, M 1..64):
+  // best at about 10 K blocks per CTA once at least ~0.8 CTA per SM stream,
+  // and no more than two CTAs per SM (the decode variants fit two).  Smallest
+  // K split (cluster size) that meets both, else the largest that fits.
+  int best = 1;
+  for (int s = 1; s <= 8 && s <= KB; ++s) {
+    const int ctas = n_tiles * s;
+    if (ctas > 2 * num_sms) break;
+    best = s;
+    if (ctas * 5 >= num_sms * 4 && (KB + s - 1) / s <= 11) break;
+  }
+  return best;
+}
+
 GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimits *limits) {
   // W4 at decode-sized M: expanded weights in tensor memory (measured 1.4x
   // faster than the smem operand at M = 16; slower at M = 2048, where the
   // smem x smem kernel below keeps W4)
   if (mode == 1 && M <= 64) return plan_gemm_w4ts(M, N, K, num_sms);
   if (M <= 64) {
-    // Decode-sized M is latency bound: a CTA streams one 16 KB weight stage
-    // per ~0.4 us whatever the tile width (measured), so what matters is how
-    // many CTAs stream at once.  128-wide tiles, K split into the smallest
-    // cluster that brings the CTA count to about one per SM, never past
-    // 1.25 per SM (a small-M CTA leaves room for a second one on its SM).
     (void)limits;
-    const int KB = K / kBlockK;
-    const int n_tiles = N / 128;
-    int best_s = 1;
-    for (int s = 1; s <= 8 && s <= KB; ++s) {
-      const int ctas = n_tiles * s;
-      if (ctas > num_sms + num_sms / 4) break;
-      best_s = s;
-      if (ctas * 5 >= num_sms * 4) break;
-    }
-    return GemmPlan{128, best_s, n_tiles * best_s, 1};
+    const int split = decode_split(N / 128, K / kBlockK, num_sms);
+    return GemmPlan{128, split, N / 128 * split, 1};
   }
   // Time model (microseconds at ~1.9 GHz).  CTAs run in waves; a wave holds
   // at most max_active(split) clusters of `split` CTAs (one CTA per SM; two for

@@ -256,9 +256,6 @@ __global__ void __launch_bounds__(kTsThreads, TsCfg<SM>::kMinBlocks)
     tmem_alloc(tmem_holder, C::kTmemCols);
     tmem_relinquish();
   }
-  if (!RAW && (warp == 2 || warp == 3)) {
-    for (int i = threadIdx.x - 64; i < 128; i += 64) s_sw[i] = p.s_w[n0 + i];
-  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -367,6 +364,9 @@ __global__ void __launch_bounds__(kTsThreads, TsCfg<SM>::kMinBlocks)
     }
   } else if ((warp == 2 || warp == 3) && !RAW) {
     // ------------------------------------ token scales of the tile, early
+    // weight scales (independent of the preceding kernel), then token
+    // scales, during the mainloop rather than on the set-up path
+    for (int i = threadIdx.x - 64; i < 128; i += 64) s_sw[i] = p.s_w[n0 + i];
     griddep_wait();
     for (int i = threadIdx.x - 64; i < bt; i += 64) s_sx[i] = m0 + i < p.M ? p.s_x[m0 + i] : 0.f;
   } else if (warp >= 4) {
@@ -704,18 +704,8 @@ GemmPlan plan_gemm_w4ts(int M, int N, int K, int num_sms) {
   const int KB = K / kBlockK;
   const int n_tiles = N / 128;
   if (M <= 64) {
-    // Decode-sized M is bound by how many CTAs stream weights at once: split
-    // K over the smallest cluster that brings the CTA count to about one per
-    // SM, never past 1.25 per SM (the two-CTA variant leaves room on the SM
-    // for a CTA of the next kernel).
-    int best_s = 1;
-    for (int s = 1; s <= 8 && s <= KB; ++s) {
-      const int ctas = n_tiles * s;
-      if (ctas > num_sms + num_sms / 4) break;
-      best_s = s;
-      if (ctas * 5 >= num_sms * 4) break;
-    }
-    return GemmPlan{128, best_s, n_tiles * best_s, 1, 1};
+    const int split = decode_split(n_tiles, KB, num_sms);
+    return GemmPlan{128, split, n_tiles * split, 1, 1};
   }
   const int m_tiles = (M + 127) / 128;
   const int ctas = m_tiles * n_tiles;

@@ -78,6 +78,8 @@ struct GemmArgs {
 cudaError_t launch_gemm(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
                         const char **why);
 GemmPlan plan_gemm_w4ts(int M, int N, int K, int num_sms);
+// K split of a decode-sized (M <= 64) launch of n_tiles 128-channel tiles.
+int decode_split(int n_tiles, int KB, int num_sms);
 cudaError_t launch_gemm_w4ts(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
                              const char **why);
 
