@@ -30,9 +30,8 @@
 namespace mixq {
 namespace {
 
-constexpr int kRowThreads = 256;  // threads per token group
-constexpr int kRowWarps = kRowThreads / 32;
-constexpr int kMaxClusterCtas = 8;
+constexpr int kRowThreads = 256;  // threads per token group, bandwidth-bound shapes
+constexpr int kMaxClusterCtas = 16;  // non-portable cluster size (opted in per kernel)
 
 __global__ void reset_detect_kernel(uint32_t *__restrict__ bitmap, int words,
                                     int32_t *__restrict__ flags) {
@@ -77,8 +76,13 @@ struct QArgs {
   int cluster_mode;  // one cluster covers the whole grid
 };
 
-template <int VPT, int G>
-__global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArgs a) {
+// RT threads per token group (256 for bandwidth-bound shapes; 512 or 1024
+// for decode-sized M, where each group handles one token and the time is the
+// latency of one token's pass), G groups per CTA, VPT 16-byte vectors per
+// thread.
+template <int VPT, int G, int RT>
+__global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
+  constexpr int kRowWarps = RT / 32;
   extern __shared__ uint32_t qsm[];
   const int words = a.K >> 5;  // K % 128 == 0
   uint32_t *s_mask = qsm;               // outlier channel bitset
@@ -89,7 +93,7 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
   __shared__ uint32_t s_mixed_total;  // cluster mode: rank 0 accumulates every CTA's count
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int g = tid / kRowThreads, gt = tid % kRowThreads, gw = gt >> 5;
+  const int g = tid / RT, gt = tid % RT, gw = gt >> 5;
   const int nvec = a.K >> 3;  // 8 fp16 per 16-byte vector
   const int row_stride = gridDim.x * G;
 
@@ -100,7 +104,7 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
   uint4 v[VPT];
 #pragma unroll
   for (int i = 0; i < VPT; ++i) {
-    const int vi = gt + i * kRowThreads;
+    const int vi = gt + i * RT;
     v[i] = (m < a.M && vi < nvec)
                ? __ldg(reinterpret_cast<const uint4 *>(a.X + static_cast<size_t>(m) * a.ldx) + vi)
                : make_uint4(0u, 0u, 0u, 0u);
@@ -154,7 +158,7 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
   auto load_row = [&](int row, uint4 *dst, int count) {
 #pragma unroll
     for (int i = 0; i < count; ++i) {
-      const int vi = gt + i * kRowThreads;
+      const int vi = gt + i * RT;
       dst[i] = (row < a.M && vi < nvec)
                    ? __ldg(reinterpret_cast<const uint4 *>(a.X + static_cast<size_t>(row) * a.ldx) +
                            vi)
@@ -168,7 +172,7 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
     float aI = 0.f, aN = 0.f;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-      const int vi = gt + i * kRowThreads;
+      const int vi = gt + i * RT;
       const int k0 = vi << 3;
       const uint32_t mb = vi < nvec ? (s_mask[k0 >> 5] >> (k0 & 31)) & 0xFFu : 0u;
       const __half2 *h = reinterpret_cast<const __half2 *>(&v[i]);
@@ -190,14 +194,14 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
       s_red[g][0][gw] = aI;
       s_red[g][1][gw] = aN;
     }
-    named_barrier(1 + g, kRowThreads);
+    named_barrier(1 + g, RT);
     float rI = s_red[g][0][0], rN = s_red[g][1][0];
 #pragma unroll
     for (int w = 1; w < kRowWarps; ++w) {
       rI = fmaxf(rI, s_red[g][0][w]);
       rN = fmaxf(rN, s_red[g][1][w]);
     }
-    named_barrier(1 + g, kRowThreads);  // s_red is rewritten by the group's next token
+    named_barrier(1 + g, RT);  // s_red is rewritten by the group's next token
 
     const float amax = fmaxf(rI, rN);
     const bool mixed = a.K_out > 0 && amax > a.T;
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
     __half *orow = a.X_out + static_cast<size_t>(m) * a.K_out_pad;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
-      const int vi = gt + i * kRowThreads;
+      const int vi = gt + i * RT;
       if (vi >= nvec) continue;
       const int k0 = vi << 3;
       const uint32_t word = s_mask[k0 >> 5];
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
       }
     }
     // every other X_out column of this token is zero
-    for (int j = gt; j < a.K_out_pad; j += kRowThreads)
+    for (int j = gt; j < a.K_out_pad; j += RT)
       if (!mixed || j >= a.K_out) orow[j] = __ushort_as_half(0);
     if (kPrefetch) {
 #pragma unroll
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
   // ------------------------------------------- matrix-wide bitmap and flags
   if (lane == 0) s_cnt[warp] = 0;
   __syncwarp();
-  if ((tid % kRowThreads) == 0) s_cnt[warp] = mixed_rows;
+  if (gt == 0) s_cnt[warp] = mixed_rows;
   __syncthreads();
   if (tid == 0) {
     int t = 0;
@@ -330,16 +334,18 @@ __global__ void __launch_bounds__(kRowThreads *G) quantize_act_kernel(const QArg
   }
 }
 
-template <int VPT, int G>
+template <int VPT, int G, int RT>
 cudaError_t launch_variant(const QArgs &a, int grid, int cluster, cudaStream_t stream) {
-  auto kernel = quantize_act_kernel<VPT, G>;
+  auto kernel = quantize_act_kernel<VPT, G, RT>;
   const size_t smem = sizeof(uint32_t) * 3 * (a.K / 32);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem < 48 * 1024 ? 48 * 1024 : smem));
+  if (e == cudaSuccess && cluster > 8)
+    e = cudaFuncSetAttribute(kernel, cudaFuncAttributeNonPortableClusterSizeAllowed, 1);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid, 1, 1);
-  cfg.blockDim = dim3(kRowThreads * G, 1, 1);
+  cfg.blockDim = dim3(RT * G, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
   cudaLaunchAttribute attr[2];
@@ -377,24 +383,25 @@ cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int3
   a.bitmap = bitmap;
   a.flags = flags;
   a.status = status;
-  const int vpt_need = (K / 8 + kRowThreads - 1) / kRowThreads;
-  const int vpt = vpt_need <= 1 ? 1 : vpt_need <= 2 ? 2 : vpt_need <= 4 ? 4 : vpt_need <= 8 ? 8 : 16;
-  // One cluster of up to 8 CTAs when that covers every token with at most 4
-  // tokens per group; G = 2 groups per CTA (1 when a row needs many
-  // registers), small enough to share an SM with a GEMM CTA.
-  const int G = vpt <= 4 ? 2 : 1;
-  const int ctas_for_m = (M + G - 1) / G;
-  if (M > 0 && ctas_for_m <= 4 * kMaxClusterCtas) {
-    const int grid = ctas_for_m < kMaxClusterCtas ? ctas_for_m : kMaxClusterCtas;
-    a.cluster_mode = 1;
-    switch (vpt) {
-      case 1: return launch_variant<1, 2>(a, grid, grid, stream);
-      case 2: return launch_variant<2, 2>(a, grid, grid, stream);
-      case 4: return launch_variant<4, 2>(a, grid, grid, stream);
-      case 8: return launch_variant<8, 1>(a, grid, grid, stream);
-      default: return launch_variant<16, 1>(a, grid, grid, stream);
+  const int nvec = K / 8;
+  if (M > 0 && M <= 64) {
+    // Decode-sized M: one token per group and wide groups (the kernel's time
+    // is one token's latency chain, measured: a second token per group adds
+    // 2-4 us), all groups in one cluster when that takes at most 16 CTAs (no
+    // reset pass, no atomics).
+    if (nvec <= 512 && (M + 1) / 2 <= kMaxClusterCtas) {  // K <= 4096: 2 x 512 threads
+      a.cluster_mode = 1;
+      return launch_variant<1, 2, 512>(a, (M + 1) / 2, (M + 1) / 2, stream);
+    }
+    if (nvec > 512 && nvec <= 2048 && M <= kMaxClusterCtas) {  // K <= 16384: 1024 threads
+      a.cluster_mode = 1;
+      return launch_variant<2, 1, 1024>(a, M, M, stream);
     }
   }
+  // Otherwise one token per 256-thread CTA at a time (grid-stride over tokens)
+  // and VPT vectors per thread.
+  const int vpt_need = (nvec + kRowThreads - 1) / kRowThreads;
+  const int vpt = vpt_need <= 1 ? 1 : vpt_need <= 2 ? 2 : vpt_need <= 4 ? 4 : vpt_need <= 8 ? 8 : 16;
   // Reset pass (waits for the preceding grid itself), then the main pass.
   {
     cudaLaunchConfig_t cfg{};
@@ -412,11 +419,11 @@ cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int3
   a.cluster_mode = 0;
   const int grid = M < num_sms * 8 ? M : num_sms * 8;
   switch (vpt) {
-    case 1: return launch_variant<1, 1>(a, grid, 1, stream);
-    case 2: return launch_variant<2, 1>(a, grid, 1, stream);
-    case 4: return launch_variant<4, 1>(a, grid, 1, stream);
-    case 8: return launch_variant<8, 1>(a, grid, 1, stream);
-    default: return launch_variant<16, 1>(a, grid, 1, stream);
+    case 1: return launch_variant<1, 1, kRowThreads>(a, grid, 1, stream);
+    case 2: return launch_variant<2, 1, kRowThreads>(a, grid, 1, stream);
+    case 4: return launch_variant<4, 1, kRowThreads>(a, grid, 1, stream);
+    case 8: return launch_variant<8, 1, kRowThreads>(a, grid, 1, stream);
+    default: return launch_variant<16, 1, kRowThreads>(a, grid, 1, stream);
   }
 }
 
