@@ -106,10 +106,13 @@ def load_peaks():
 
 
 def kernel_source_hash() -> str:
+    """Hash of every kernel source file: committed ncu counters apply only to these sources."""
     h = hashlib.sha256()
-    for f in ("gemm.cu", "quantize.cu", "ptx.cuh", "internal.h"):
-        with open(os.path.join(ROOT, "mixed_precision_quantized_mixq_b200", "csrc", f), "rb") as fh:
-            h.update(fh.read())
+    csrc = os.path.join(ROOT, "mixed_precision_quantized_mixq_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if f.endswith((".cu", ".cuh", ".h")):
+            with open(os.path.join(csrc, f), "rb") as fh:
+                h.update(f.encode() + b"\0" + fh.read())
     return h.hexdigest()[:16]
 
 

@@ -109,6 +109,13 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
                ? __ldg(reinterpret_cast<const uint4 *>(a.X + static_cast<size_t>(m) * a.ldx) + vi)
                : make_uint4(0u, 0u, 0u, 0u);
   }
+  // The first outlier index of this thread is read alongside the token row
+  // (both latencies overlap); any further ones below.
+  int c_first = -1, c_prev = -1;
+  if (tid < a.K_out) {
+    c_first = a.idx[tid];
+    c_prev = tid > 0 ? a.idx[tid - 1] : -1;
+  }
   for (int w = tid; w < words; w += blockDim.x) {
     s_mask[w] = 0u;
     s_det[w] = 0u;
@@ -122,8 +129,9 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   // matching wait comes before any CTA adds into rank 0's
   if (a.cluster_mode) cluster_arrive_relaxed();
   for (int j = tid; j < a.K_out; j += blockDim.x) {
-    const int c = a.idx[j];
-    const bool ok = c >= 0 && c < a.K && (j == 0 || a.idx[j - 1] < c);
+    const int c = j == tid ? c_first : a.idx[j];
+    const int cp = j == tid ? c_prev : a.idx[j - 1];
+    const bool ok = c >= 0 && c < a.K && (j == 0 || cp < c);
     if (!ok) s_bad = 1;
     else atomicOr(&s_mask[c >> 5], 1u << (c & 31));
   }
@@ -417,6 +425,8 @@ cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int3
     if (e != cudaSuccess || M == 0) return e;
   }
   a.cluster_mode = 0;
+  if (M <= 64 && nvec <= 512) return launch_variant<1, 2, 512>(a, (M + 1) / 2, 1, stream);
+  if (M <= 64 && nvec <= 2048) return launch_variant<2, 1, 1024>(a, M, 1, stream);
   const int grid = M < num_sms * 8 ? M : num_sms * 8;
   switch (vpt) {
     case 1: return launch_variant<1, 1, kRowThreads>(a, grid, 1, stream);
