@@ -12,9 +12,12 @@ weight copies, so a step touches more bytes than the 126 MB L2 and nothing is
 served from L2 across steps.
 
 The step is captured once in a CUDA graph (decode-sized kernels run for a few
-microseconds, shorter than their host launch cost) and replayed; CUDA events
-recorded inside the graph time each kernel, events around the replays time the
-steps.  Prints ONE JSON line on rank 0.
+microseconds, shorter than their host launch cost) and replayed; events around
+the replays time the steps.  Copies of the graph with events at the phase
+boundaries (quantize / W8A8 / W4A8), replayed right after, time each kernel
+kind.  The end-to-end leg moves every step's inputs in from pinned host memory
+and its outputs back, overlapping neighbouring steps' copies with the kernels.
+Prints ONE JSON line on rank 0.
 
 --impl reference times the CPU oracle (the plain C restatement of the layer)
 on the host cores as the reference arm, on a bounded sample of the same
@@ -103,6 +106,15 @@ def load_peaks():
         return {k: float(d[k]) for k in FALLBACK_PEAKS}, "measured"
     except Exception:
         return dict(FALLBACK_PEAKS), "fallback"
+
+
+def quantize_launches(M: int, K: int) -> int:
+    """Kernels one mixq_quantize_act call launches: one cluster for decode-sized M
+    (at most 16 CTAs of 1024 threads), else a reset pass and the main pass."""
+    nvec = K // 8
+    if 0 < M <= 64 and ((nvec <= 512 and (M + 1) // 2 <= 16) or (512 < nvec <= 2048 and M <= 16)):
+        return 1
+    return 2
 
 
 def kernel_source_hash() -> str:
@@ -243,17 +255,24 @@ def run_gpu(args, rank, world):
     y_sizes = [L["case"].M * L["case"].N * len(L["modes"]) for L in layers]
     X_all = torch.empty(sum(x_sizes), dtype=torch.float16, device=dev)
     Y_all = torch.empty(sum(y_sizes), dtype=torch.float16, device=dev)
-    xo = yo = 0
-    for L, xs, ys in zip(layers, x_sizes, y_sizes):
-        c = L["case"]
-        L["X"] = X_all[xo:xo + xs].view(c.M, c.K)
-        L["X"].copy_(torch.from_numpy(L.pop("Xh")))
-        L["Y"] = {}
-        for mi, m in enumerate(L["modes"]):
-            L["Y"][m] = Y_all[yo + mi * c.M * c.N: yo + (mi + 1) * c.M * c.N].view(c.M, c.N)
-        L["q"] = mq.quantize_act(L["X"], L["idx"], T)
-        xo += xs
-        yo += ys
+
+    def bind(Xb, Yb):
+        """Per-case views (X, Y per mode) of one packed activation/output buffer pair."""
+        views, xo, yo = [], 0, 0
+        for L, xs, ys in zip(layers, x_sizes, y_sizes):
+            c = L["case"]
+            V = {"X": Xb[xo:xo + xs].view(c.M, c.K), "Y": {}}
+            for mi, m in enumerate(L["modes"]):
+                V["Y"][m] = Yb[yo + mi * c.M * c.N: yo + (mi + 1) * c.M * c.N].view(c.M, c.N)
+            views.append(V)
+            xo += xs
+            yo += ys
+        return views
+
+    views0 = bind(X_all, Y_all)
+    for L, V in zip(layers, views0):
+        V["X"].copy_(torch.from_numpy(L.pop("Xh")))
+        V["q"] = mq.quantize_act(V["X"], L["idx"], T)
     torch.cuda.synchronize()
 
     status = torch.zeros(1, dtype=torch.int32, device=dev)
@@ -264,20 +283,21 @@ def run_gpu(args, rank, world):
             if m not in modes_all:
                 modes_all.append(m)
 
-    def step(events=None):
+    def step(events=None, views=None):
         # Phase order: every case's quantize, then every case's W8A8 GEMM, then
         # every W4A8 GEMM.  Timing events sit only at the phase boundaries, so
         # consecutive kernels keep overlapping (programmatic dependent launch).
+        views = views0 if views is None else views
         if events is not None:
             events[0].record()
-        for L in layers:
-            mq.quantize_act(L["X"], L["idx"], T, out=L["q"], status=status)
+        for L, V in zip(layers, views):
+            mq.quantize_act(V["X"], L["idx"], T, out=V["q"], status=status)
         if events is not None:
             events[1].record()
         for mi, m in enumerate(modes_all):
-            for L in layers:
+            for L, V in zip(layers, views):
                 if m in L["modes"]:
-                    mq.gemm(L["q"], L["packed"][m], Y=L["Y"][m], status=status)
+                    mq.gemm(V["q"], L["packed"][m], Y=V["Y"][m], status=status)
             if events is not None:
                 events[2 + mi].record()
 
@@ -286,13 +306,18 @@ def run_gpu(args, rank, world):
         step()
     torch.cuda.synchronize()
     mq.check_status(status)
-    mixed = [int(L["q"].flags[0].item()) > 0 for L in layers]
+    mixed = [int(V["q"].flags[0].item()) > 0 for V in views0]
 
-    # ---- up to 32 CUDA graphs of one step each, replayed round-robin; each has its own
-    # timing events, so after the timed region every graph's events hold the kernel
-    # durations of its last replay (the last n_graphs steps of the timed region)
-    n_graphs = min(args.steps, 32)
+    # ---- the step as one CUDA graph (the timed region of the whole-step value), and
+    # up to 32 copies with timing events at the phase boundaries, replayed once each
+    # right after it: their events give the per-kernel-kind durations.  (Event nodes
+    # inside a graph cost the chained kernels some of their overlap, about 5 % of a
+    # decode step, so they stay out of the value's timed region.)
     side = torch.cuda.Stream(device=dev)
+    g_step = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_step, stream=side):
+        step()
+    n_graphs = min(args.steps, 32)
     graphs, ev_sets = [], []
     for g_i in range(n_graphs):
         evs = [torch.cuda.Event(enable_timing=True, external=True)
@@ -305,7 +330,7 @@ def run_gpu(args, rank, world):
     torch.cuda.synchronize()
 
     for i in range(args.warmup):
-        graphs[i % n_graphs].replay()
+        g_step.replay()
     torch.cuda.synchronize()
 
     gpu_id = None
@@ -324,8 +349,10 @@ def run_gpu(args, rank, world):
     sampler.mark(True)
     start.record()
     for i in range(args.steps):
-        graphs[i % n_graphs].replay()
+        g_step.replay()
     end.record()
+    for g in graphs:
+        g.replay()
     torch.cuda.synchronize()
     sampler.mark(False)
     if world > 1:
@@ -384,30 +411,64 @@ def run_gpu(args, rank, world):
                  "share_of_step": {k: round(v[0] / max(1e-9, sum(x[0] for x in kinds.values())), 4)
                                    for k, v in kinds.items()}})
 
-    # ---- end to end: host X in pinned memory -> device -> layer -> Y back to pinned host
+    # ---- end to end: host X in pinned memory -> device -> layer -> Y back to pinned host.
+    # Every step copies its inputs in and its outputs out; two device buffer sets
+    # let step i+1's input copy and step i-1's output copy run beside step i's
+    # kernels (three streams, ordered by events).
     host_X = X_all.cpu().pin_memory()
     host_Y = torch.empty(Y_all.shape, dtype=torch.float16).pin_memory()
     h2d = host_X.numel() * 2
     d2h = host_Y.numel() * 2
+    X_all1, Y_all1 = torch.empty_like(X_all), torch.empty_like(Y_all)
+    views1 = bind(X_all1, Y_all1)
+    X_all1.copy_(X_all)
+    for L, V in zip(layers, views1):
+        V["q"] = mq.quantize_act(V["X"], L["idx"], T)
+    torch.cuda.synchronize()
+    bufX, bufY = (X_all, X_all1), (Y_all, Y_all1)
+    ge = []
+    for views in (views0, views1):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=side):
+            step(views=views)
+        ge.append(g)
+    s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+    ev_in = [torch.cuda.Event() for _ in range(2)]
+    ev_comp = [torch.cuda.Event() for _ in range(2)]
+    ev_out = [torch.cuda.Event() for _ in range(2)]
 
-    def e2e_step():
-        X_all.copy_(host_X, non_blocking=True)
-        step()
-        host_Y.copy_(Y_all, non_blocking=True)
+    def run_e2e(n, start_ev=None, end_ev=None):
+        if start_ev is not None:
+            start_ev.record(s_in)
+        with torch.cuda.stream(s_in):
+            bufX[0].copy_(host_X, non_blocking=True)
+            ev_in[0].record(s_in)
+        for i in range(n):
+            b = i % 2
+            if i + 1 < n:  # next step's input, once step i-1 is done reading that buffer
+                nb = (i + 1) % 2
+                s_in.wait_event(ev_comp[nb])
+                with torch.cuda.stream(s_in):
+                    bufX[nb].copy_(host_X, non_blocking=True)
+                    ev_in[nb].record(s_in)
+            side.wait_event(ev_in[b])
+            side.wait_event(ev_out[b])  # step i-2's output copy is out of Y[b]
+            with torch.cuda.stream(side):
+                ge[b].replay()
+                ev_comp[b].record(side)
+            s_out.wait_event(ev_comp[b])
+            with torch.cuda.stream(s_out):
+                host_Y.copy_(bufY[b], non_blocking=True)
+                ev_out[b].record(s_out)
+        if end_ev is not None:
+            end_ev.record(s_out)
 
-    ge = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(ge, stream=side):
-        e2e_step()
-    for _ in range(max(3, args.warmup)):
-        ge.replay()
+    run_e2e(max(3, args.warmup))
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     s2, e2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    s2.record()
-    for _ in range(args.steps):
-        ge.replay()
-    e2.record()
+    run_e2e(args.steps, s2, e2)
     torch.cuda.synchronize()
     e2e_ms = s2.elapsed_time(e2)
     e2e_ms = max_over_ranks(e2e_ms, world, dev)
@@ -415,12 +476,12 @@ def run_gpu(args, rank, world):
     e2e = {"value": round(ops_step * world / (e2e_ms / args.steps * 1e-3) / 1e12, 4),
            "unit": "TOPS", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
            "ms_per_step": round(e2e_ms / args.steps, 5),
-           "how": "one pinned-host -> device copy of every case's X, quantize + both GEMMs, one "
-                  "device -> pinned-host copy of every Y; CUDA graph"}
+           "how": "per step: one pinned-host -> device copy of every case's X, quantize + both "
+                  "GEMMs (CUDA graph), one device -> pinned-host copy of every Y; copies of "
+                  "neighbouring steps overlap the kernels (two device buffer sets, three streams)"}
 
-    # quantize is one kernel for decode-sized M (one cluster), else reset + main pass
-    launches_per_step = sum((1 if L["case"].M <= (64 if L["case"].K <= 8192 else 32) else 2)
-                            + len(L["modes"]) for L in layers)
+    launches_per_step = sum(quantize_launches(L["case"].M, L["case"].K) + len(L["modes"])
+                            for L in layers)
     touched = sum(L["packed"][m].Wq.numel() * L["packed"][m].Wq.element_size()
                   for L in layers for m in L["modes"])
     result = {
@@ -430,12 +491,14 @@ def run_gpu(args, rank, world):
         "dtype": "int8 (int8 x int8 -> int32 tensor cores) + fp16 outlier slice (fp32 accumulate)",
         "data": "synthetic (seeded normals; random-init weights of the Llama shapes)",
         "config": {"workload": args.workload, "description": desc, "cases": len(layers),
-                   "mixed_tokens_per_case": [int(L["q"].flags[0].item()) for L in layers],
+                   "mixed_tokens_per_case": [int(V["q"].flags[0].item()) for V in views0],
                    "l2": f"inputs larger than L2: {touched / 1e6:.0f} MB of distinct weights per "
                          "step (126 MB L2), each case reads its own copy",
                    "launch": "one CUDA graph per step (captured once, replayed); kernels chained "
                              "with programmatic dependent launch; step order: all quantize, "
-                             "all W8A8 GEMMs, all W4A8 GEMMs; timing events at phase boundaries",
+                             "all W8A8 GEMMs, all W4A8 GEMMs; per-kernel-kind times from "
+                             "graph copies with events at the phase boundaries, replayed after "
+                             "the timed steps",
                    "parallelism": f"dp{world} (independent batches per GPU, no collective)"},
         "roofline": roof,
         "e2e": e2e,
