@@ -385,10 +385,22 @@ __global__ void __launch_bounds__(kTsThreads, TsCfg<SM>::kMinBlocks)
         ok = false;
         break;
       }
+      // expand both K blocks of the job first (independent work for the
+      // scheduler), release the codes, and only then wait for the A stage
+      const uint8_t *sp = stage(s);
+      const int nkb = job_nkb(j);
+      uint32_t wv0[32], wv1[32];
+      expand_chunks<4>(sp, sp + kbpj * kTsPacked, row, psw, 0, wv0);
+      if (nkb == 2) expand_chunks<4>(sp + kTsPacked, sp + kbpj * kTsPacked + kTsGrp, row, psw, 0, wv1);
+      // the codes are consumed: the stage's weight half is free (one arrival
+      // per warp)
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      r.advance(stages);
       if (j >= p.a_stages) {
         // A stage j % a_stages was last read by job j - a_stages, whose commit
         // completes that job's phase of empty[].  (stages >= a_stages keeps the
-        // phase unambiguous: this warp's arrival for the slot's next use comes
+        // phase unambiguous: this warp's arrival for that slot's next use comes
         // only after the producer refilled it, i.e. after that phase.)
         if (!warp_wait(&empty[rf.slot], rf.phase, p.wait_limit_ns)) {
           ok = false;
@@ -397,21 +409,9 @@ __global__ void __launch_bounds__(kTsThreads, TsCfg<SM>::kMinBlocks)
         rf.advance(stages);
       }
       tc_fence_after();
-      const uint8_t *sp = stage(s);
       const uint32_t ta = t_a + lane_addr + ra.slot * a_cols;
-      // every K block of the job: 4 chunks -> 32 TMEM columns each
-      const int nkb = job_nkb(j);
-      for (int kk = 0; kk < nkb; ++kk) {
-        uint32_t wv[32];
-        expand_chunks<4>(sp + kk * kTsPacked, sp + kbpj * kTsPacked + kk * kTsGrp, row, psw, 0,
-                         wv);
-        tmem_st32(ta + kk * 32, wv);
-      }
-      // the codes are consumed: the stage's weight half is free (one arrival
-      // per warp)
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&empty[s]);
-      r.advance(stages);
+      tmem_st32(ta, wv0);
+      if (nkb == 2) tmem_st32(ta + 32, wv1);
       tmem_st_wait();
       tc_fence_before();
       __syncwarp();
