@@ -205,9 +205,9 @@ static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const i
   a.epi = mixq::Epi::kMixed;
   a.status = status;
   a.wait_limit_ns = kDefaultWaitNs;
-  // (the decode-sized W4 planner needs no occupancy table)
+  // (the W4 planner below M = 1024 needs no occupancy table)
   const mixq::GemmPlan plan = mixq::plan_gemm(
-      mode, M, N, K, sms, (mode == MIXQ_W8 || M > 64) ? mixq::device_cluster_limits(mode) : nullptr);
+      mode, M, N, K, sms, (mode == MIXQ_W8 || M > 1024) ? mixq::device_cluster_limits(mode) : nullptr);
   const char *why = nullptr;
   const cudaError_t e = mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why);
   return from_cuda(e, "gemm launch", why);
@@ -286,7 +286,7 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   s = check_device(&sms);
   if (s != MIXQ_OK) return s;
   mixq::GemmPlan plan = mixq::plan_gemm(
-      mode, M, N, K, sms, (mode == MIXQ_W8 || M > 64) ? mixq::device_cluster_limits(mode) : nullptr);
+      mode, M, N, K, sms, (mode == MIXQ_W8 || M > 1024) ? mixq::device_cluster_limits(mode) : nullptr);
   if (split) plan.split = split;
   if (mode == MIXQ_W4G128 && (bn == 128 || bn == 256 || (bn == 0 && plan.ts))) {
     // tensor-memory-operand kernel: bn = 128 the two-CTA-per-SM variant,
