@@ -125,6 +125,19 @@ def quantize_act(X: np.ndarray, idx, T: float):
     return Xq, s_x, X_out.view(np.float16), bitmap, flags
 
 
+def rmsnorm(X: np.ndarray, g: np.ndarray, eps: float) -> np.ndarray:
+    """RMS-normalised tokens Y = fp16(X / sqrt(mean(X^2) + eps) * g), fp64 inside."""
+    lib = _load()
+    M, K = X.shape
+    Y = np.empty((M, K), np.uint16)
+    lib.oracle_rmsnorm.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                   ctypes.c_void_p, ctypes.c_double, ctypes.c_void_p]
+    rc = lib.oracle_rmsnorm(_p(_f16bits(X)), M, K, K, _p(_f16bits(np.asarray(g, np.float16))),
+                            float(eps), _p(Y))
+    _check(rc, "rmsnorm")
+    return Y.view(np.float16)
+
+
 def gemm_i32(Xq: np.ndarray, Wq: np.ndarray, m0: int = 0, m1: int | None = None):
     """Exact INT32 accumulators acc[m,n] = sum_k Xq[m,k]*Wq[n,k] for rows [m0,m1)."""
     lib = _load()

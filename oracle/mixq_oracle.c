@@ -185,6 +185,38 @@ int oracle_prepack_w4(const int8_t *Wq8, int N, int K, uint8_t *q, uint8_t *s2, 
 }
 
 /*
+ * RMS normalisation of each token: the operation before the layer, which the
+ * activation pass can absorb ([MixQ] MixQ的解决方案: the amax of quantization
+ * can be taken inside the preceding operation).  The pages give no formula for
+ * that operation; reading: the Llama RMSNorm
+ *   Y[m,k] = fp16( X[m,k] / sqrt(mean_k X[m,k]^2 + eps) * g[k] ),
+ * evaluated in fp64 (sum, mean, square root, division, both products) and
+ * rounded once to fp16, round to nearest even.
+ *   X [M][ldx] fp16 bits, g [K] fp16 bits, eps >= 0, Y [M][K] fp16 bits.
+ */
+int oracle_rmsnorm(const uint16_t *X, int M, int K, int ldx, const uint16_t *g, double eps,
+                   uint16_t *Y) {
+  if (M < 0 || K <= 0 || ldx < K || !(eps >= 0.0) || !isfinite(eps)) return ORC_EINVAL;
+  for (int k = 0; k < K; ++k)
+    if (!isfinite(h2f(g[k]))) return ORC_ENONFINITE;
+  for (int m = 0; m < M; ++m) {
+    const uint16_t *x = X + (size_t)m * ldx;
+    double ss = 0.0;
+    for (int k = 0; k < K; ++k) {
+      double v = (double)h2f(x[k]);
+      if (!isfinite(v)) return ORC_ENONFINITE;
+      ss += v * v;
+    }
+    double den = sqrt(ss / (double)K + eps);
+    for (int k = 0; k < K; ++k) {
+      double v = den > 0.0 ? (double)h2f(x[k]) / den * (double)h2f(g[k]) : 0.0;
+      Y[(size_t)m * K + k] = f2h_bits(v);
+    }
+  }
+  return ORC_OK;
+}
+
+/*
  * Activation quantization with outlier detection ([MixQ] MixQ的解决方案: the
  * amax taken for quantization tells whether outliers exist -- amax greater
  * than the threshold means yes; Fig. 10 equivalent transformation

@@ -345,3 +345,46 @@ def test_round_f16_nearest_even():
     got = oracle.round_f16(v)
     np.testing.assert_array_equal(got.astype(np.float64), [1.0, 1.0 + 2.0 ** -9, 65504.0, -0.0,
                                                             np.float16(6.0e-8)])
+
+
+# ------------------------------------------------- RMS normalisation (next row f1)
+def test_rmsnorm_golden_cases(golden_dir):
+    g = _load(golden_dir, "rmsnorm_cases.json")
+    for c in g["cases"]:
+        X = np.asarray([c["x"]], np.float16)
+        y = oracle.rmsnorm(X, np.asarray(c["g"], np.float16), c["eps"])
+        assert y.view(np.uint16)[0].tolist() == c["y_bits"], c["name"]
+
+
+def test_rmsnorm_scale_invariance_and_gain():
+    # eps = 0: scaling a token by a power of two changes nothing, and scaling the
+    # gain by a power of two scales the output exactly (as long as every scaled
+    # value stays a normal fp16 number, so the scaling itself is exact)
+    X = synth.activations(6, 512)
+    g = np.random.default_rng(7).normal(1.0, 0.1, 512).astype(np.float16)
+    y = oracle.rmsnorm(X, g, 0.0)
+    assert np.abs(X[X != 0]).min() * 0.5 >= 2.0 ** -14 and np.abs(X).max() * 4 < 65504
+    for j in (-1, 2):
+        Xs = (X.astype(np.float32) * 2.0 ** j).astype(np.float16)
+        assert np.array_equal(oracle.rmsnorm(Xs, g, 0.0).view(np.uint16), y.view(np.uint16))
+    g2 = (g.astype(np.float32) * 2.0).astype(np.float16)
+    assert np.array_equal(oracle.rmsnorm(X, g2, 0.0).astype(np.float32), 2.0 * y.astype(np.float32))
+
+
+def test_rmsnorm_unit_rms_and_eps():
+    # unit gain, eps = 0: every output row has mean square 1 (up to fp16 rounding);
+    # eps > 0 shrinks it to ms / (ms + eps)
+    X = synth.activations(8, 1024)
+    one = np.ones(1024, np.float16)
+    ms = (oracle.rmsnorm(X, one, 0.0).astype(np.float64) ** 2).mean(axis=1)
+    assert np.all(np.abs(ms - 1.0) < 2e-3)
+    x_ms = (X.astype(np.float64) ** 2).mean(axis=1)
+    eps = 0.5
+    ms_eps = (oracle.rmsnorm(X, one, eps).astype(np.float64) ** 2).mean(axis=1)
+    assert np.all(np.abs(ms_eps - x_ms / (x_ms + eps)) < 2e-3)
+
+
+def test_rmsnorm_rejects_bad_eps():
+    X = np.ones((1, 8), np.float16)
+    with pytest.raises(oracle.OracleError):
+        oracle.rmsnorm(X, np.ones(8, np.float16), -1.0)
