@@ -142,6 +142,26 @@ mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_
                               void *stream);
 
 /*
+ * The activation pass with the preceding RMS normalisation absorbed (MixQ
+ * article, MixQ的解决方案: the quantization amax can be taken inside the
+ * operation before the layer).  Per token, in fp32 with IEEE division and
+ * square root:
+ *   Xn[m,k] = fp16( X[m,k] / sqrt(mean_k X[m,k]^2 + eps) * gamma[k] )
+ * then exactly mixq_quantize_act on Xn (same outputs, same launches).  X is
+ * read once and Xn never has to go through HBM; it is written only when
+ * Xn != NULL (ldxn >= K, multiple of 8).  A row whose mean square plus eps is
+ * 0 normalises to zeros.
+ *   gamma fp16 [K] (16-byte aligned, non-null), eps finite >= 0; the other
+ *   arguments as mixq_quantize_act.  Errors: MIXQ_ERR_INVALID_ARG for a null
+ *   gamma or a bad eps/ldxn, otherwise as mixq_quantize_act.
+ */
+mixq_status mixq_rmsnorm_quantize_act(const void *X, int M, int K, int ldx, const void *gamma,
+                                      float eps, void *Xn, int ldxn, const int32_t *idx,
+                                      int K_out, float threshold, int8_t *Xq, float *s_x,
+                                      void *X_out, uint32_t *detect_bitmap, int32_t *flags,
+                                      int32_t *status, void *stream);
+
+/*
  * Mixed-precision GEMM, 8-bit weights (MixQ Fig. 5 decomposition; Fig. 12
  * fused dequantize, scale and add of the INT32 result in registers):
  *   acc[m,n] = sum_k Xq[m,k] Wq[n,k]                     (exact INT32, tcgen05 kind::i8)

@@ -32,6 +32,8 @@ _SIGNATURES = {
     "mixq_prepack_size": (_I, [_I, _I, _I, _I, _c.POINTER(_SZ), _c.POINTER(_SZ), _c.POINTER(_SZ)]),
     "mixq_prepack_weights": (_I, [_I, _VP, _I, _I, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP]),
     "mixq_quantize_act": (_I, [_VP, _I, _I, _I, _VP, _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "mixq_rmsnorm_quantize_act": (_I, [_VP, _I, _I, _I, _VP, _F, _VP, _I, _VP, _I, _F, _VP, _VP,
+                                       _VP, _VP, _VP, _VP, _VP]),
     "mixq_gemm_w8a8o16": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _VP,
                                _VP]),
     "mixq_gemm_w4a8o16": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I,
@@ -110,6 +112,16 @@ def mixq_quantize_act(X, idx, threshold, Xq, s_x, X_out, bitmap, flags, status, 
                                    0 if idx is None else idx.numel(), float(threshold), _ptr(Xq),
                                    _ptr(s_x), _ptr(X_out), _ptr(bitmap), _ptr(flags), _ptr(status),
                                    _stream(stream)))
+
+
+def mixq_rmsnorm_quantize_act(X, gamma, eps, Xn, idx, threshold, Xq, s_x, X_out, bitmap, flags,
+                              status, stream=None):
+    M, K = X.shape
+    _check(lib().mixq_rmsnorm_quantize_act(_ptr(X), M, K, X.stride(0), _ptr(gamma), float(eps),
+                                           _ptr(Xn), 0 if Xn is None else Xn.stride(0), _ptr(idx),
+                                           0 if idx is None else idx.numel(), float(threshold),
+                                           _ptr(Xq), _ptr(s_x), _ptr(X_out), _ptr(bitmap),
+                                           _ptr(flags), _ptr(status), _stream(stream)))
 
 
 def mixq_gemm_w8a8o16(M, N, K, K_out, Xq, s_x, X_out, Wq, s_w, W_out, flags, Y, status,
@@ -242,6 +254,26 @@ def quantize_act(X, idx, threshold: float = 6.0, out: QuantAct | None = None, st
                        torch.empty(4, dtype=torch.int32, device=dev))
     mixq_quantize_act(X, idx if ko else None, threshold, out.Xq, out.s_x, out.X_out, out.bitmap,
                       out.flags, status, stream)
+    return out
+
+
+def rmsnorm_quantize_act(X, gamma, eps: float, idx, threshold: float = 6.0,
+                         out: QuantAct | None = None, Xn=None, status=None,
+                         stream=None) -> QuantAct:
+    """RMS-normalise each token (gain gamma, eps) and run the activation pass on
+    the result in the same kernel; Xn (optional) receives the normalised tokens."""
+    torch = _require_cuda()
+    M, K = X.shape
+    dev = X.device
+    ko = idx.numel()
+    if out is None:
+        out = QuantAct(torch.empty((M, K), dtype=torch.int8, device=dev),
+                       torch.empty(M, dtype=torch.float32, device=dev),
+                       torch.empty((M, k_out_pad(ko)), dtype=torch.float16, device=dev) if ko else None,
+                       torch.empty(K // 32, dtype=torch.int32, device=dev),
+                       torch.empty(4, dtype=torch.int32, device=dev))
+    mixq_rmsnorm_quantize_act(X, gamma, eps, Xn, idx if ko else None, threshold, out.Xq, out.s_x,
+                              out.X_out, out.bitmap, out.flags, status, stream)
     return out
 
 

@@ -138,10 +138,11 @@ mixq_status mixq_prepack_weights(int mode, const void *W, int N, int K, const in
                    "prepack launch");
 }
 
-mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx, int K_out,
-                              float threshold, int8_t *Xq, float *s_x, void *X_out,
-                              uint32_t *detect_bitmap, int32_t *flags, int32_t *status,
-                              void *stream) {
+static mixq_status quantize_common(const void *X, int M, int K, int ldx, const int32_t *idx,
+                                   int K_out, float threshold, int8_t *Xq, float *s_x,
+                                   void *X_out, uint32_t *detect_bitmap, int32_t *flags,
+                                   int32_t *status, void *stream, const void *gamma, float eps,
+                                   void *Xn, int ldxn) {
   mixq_status s = check_shape(M, 128, K, K_out);
   if (s != MIXQ_OK) return s;
   if (K > mixq::quantize_max_k())
@@ -154,16 +155,40 @@ mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_
   if (M > 0 && (!X || !Xq || !s_x)) return fail(MIXQ_ERR_INVALID_ARG, "X, Xq and s_x must be non-null");
   if (K_out > 0 && !idx) return fail(MIXQ_ERR_INVALID_ARG, "idx must be non-null when K_out > 0");
   if (K_out > 0 && M > 0 && !X_out) return fail(MIXQ_ERR_INVALID_ARG, "X_out must be non-null when K_out > 0");
+  if (Xn && (ldxn < K || ldxn % 8))
+    return fail(MIXQ_ERR_INVALID_ARG, "ldxn = %d must be >= K and a multiple of 8", ldxn);
   if ((X && !aligned16(X)) || (Xq && !aligned16(Xq)) || (X_out && !aligned16(X_out)) ||
-      !aligned16(detect_bitmap) || !aligned16(flags))
+      !aligned16(detect_bitmap) || !aligned16(flags) || (gamma && !aligned16(gamma)) ||
+      (Xn && !aligned16(Xn)))
     return fail(MIXQ_ERR_MISALIGNED, "matrix pointers must be 16-byte aligned");
   int sms = 0;
   s = check_device(&sms);
   if (s != MIXQ_OK) return s;
   return from_cuda(mixq::launch_quantize_act(X, M, K, ldx, idx, K_out, threshold, Xq, s_x, X_out,
                                              detect_bitmap, flags, status,
-                                             static_cast<cudaStream_t>(stream), sms),
+                                             static_cast<cudaStream_t>(stream), sms, gamma, eps,
+                                             Xn, ldxn),
                    "quantize launch");
+}
+
+mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx, int K_out,
+                              float threshold, int8_t *Xq, float *s_x, void *X_out,
+                              uint32_t *detect_bitmap, int32_t *flags, int32_t *status,
+                              void *stream) {
+  return quantize_common(X, M, K, ldx, idx, K_out, threshold, Xq, s_x, X_out, detect_bitmap,
+                         flags, status, stream, nullptr, 0.f, nullptr, 0);
+}
+
+mixq_status mixq_rmsnorm_quantize_act(const void *X, int M, int K, int ldx, const void *gamma,
+                                      float eps, void *Xn, int ldxn, const int32_t *idx,
+                                      int K_out, float threshold, int8_t *Xq, float *s_x,
+                                      void *X_out, uint32_t *detect_bitmap, int32_t *flags,
+                                      int32_t *status, void *stream) {
+  if (!gamma) return fail(MIXQ_ERR_INVALID_ARG, "gamma must be non-null");
+  if (!(eps >= 0.f) || eps != eps || eps > 3.0e38f)
+    return fail(MIXQ_ERR_INVALID_ARG, "eps must be a finite value >= 0");
+  return quantize_common(X, M, K, ldx, idx, K_out, threshold, Xq, s_x, X_out, detect_bitmap,
+                         flags, status, stream, gamma, eps, Xn, ldxn);
 }
 
 static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const int8_t *Xq,

@@ -19,10 +19,12 @@ inline int k_out_pad(int k_out) { return (k_out + 63) / 64 * 64; }
 
 // ---------------------------------------------------------------- quantize
 int quantize_max_k();  // largest K the quantize kernel holds in registers
+// gamma != nullptr: RMS-normalise each token first (eps; optional Xn output).
 cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx,
                                 int K_out, float threshold, int8_t *Xq, float *s_x, void *X_out,
                                 uint32_t *bitmap, int32_t *flags, int32_t *status,
-                                cudaStream_t stream, int num_sms);
+                                cudaStream_t stream, int num_sms, const void *gamma = nullptr,
+                                float eps = 0.f, void *Xn = nullptr, int ldxn = 0);
 
 // ----------------------------------------------------------------- prepack
 cudaError_t launch_prepack(int mode, const void *W, int N, int K, const int32_t *idx, int K_out,

@@ -48,6 +48,12 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+__device__ __forceinline__ float warp_sum_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = __fadd_rn(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
 __device__ __forceinline__ int warp_sum(int v) {
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
@@ -64,6 +70,10 @@ __device__ __forceinline__ uint32_t code8(float x, float inv) {
 struct QArgs {
   const __half *X;
   int M, K, ldx;
+  const __half *gamma;  // RMS-normalisation gain [K] (NORM variants)
+  float eps;
+  __half *Xn;           // optional normalised tokens [M][ldxn] (NORM variants)
+  int ldxn;
   const int32_t *idx;
   int K_out, K_out_pad;
   float T;
@@ -79,8 +89,10 @@ struct QArgs {
 // RT threads per token group (256 for bandwidth-bound shapes; 512 or 1024
 // for decode-sized M, where each group handles one token and the time is the
 // latency of one token's pass), G groups per CTA, VPT 16-byte vectors per
-// thread.
-template <int VPT, int G, int RT>
+// thread.  NORM: the token is first RMS-normalised in registers
+// (x / sqrt(mean x^2 + eps) * gamma, rounded to fp16 as the normalisation's
+// output would be), so the pass reads X once for both operations.
+template <int VPT, int G, int RT, bool NORM>
 __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   constexpr int kRowWarps = RT / 32;
   extern __shared__ uint32_t qsm[];
@@ -177,6 +189,55 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   for (; m < a.M; m += row_stride) {
     uint4 vn[kVn];
     if (kPrefetch) load_row(m + row_stride, vn, kVn);
+    if (NORM) {
+      // mean square of the token (fp32, sequential per thread, then a
+      // shuffle tree, then the warps in order), one IEEE sqrt, and per
+      // element one IEEE division and one multiply, rounded to fp16.  The
+      // gain vectors are loaded here (cached after the first token) so their
+      // latency overlaps the reduction, without holding registers across tokens.
+      uint4 gv[VPT];
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const int vi = gt + i * RT;
+        gv[i] = vi < nvec ? __ldg(reinterpret_cast<const uint4 *>(a.gamma) + vi)
+                          : make_uint4(0u, 0u, 0u, 0u);
+      }
+      float ss = 0.f;
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const __half2 *h = reinterpret_cast<const __half2 *>(&v[i]);
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float2 f = __half22float2(h[e2]);
+          ss = __fadd_rn(ss, __fmul_rn(f.x, f.x));
+          ss = __fadd_rn(ss, __fmul_rn(f.y, f.y));
+        }
+      }
+      ss = warp_sum_f(ss);
+      if (lane == 0) s_red[g][0][gw] = ss;
+      named_barrier(1 + g, RT);
+      float tot = 0.f;
+#pragma unroll
+      for (int w = 0; w < kRowWarps; ++w) tot = __fadd_rn(tot, s_red[g][0][w]);
+      named_barrier(1 + g, RT);  // s_red is rewritten by the amax below
+      const float den = __fsqrt_rn(__fadd_rn(__fdiv_rn(tot, static_cast<float>(a.K)), a.eps));
+      __half *xn_row = a.Xn ? a.Xn + static_cast<size_t>(m) * a.ldxn : nullptr;
+#pragma unroll
+      for (int i = 0; i < VPT; ++i) {
+        const int vi = gt + i * RT;
+        __half2 *h = reinterpret_cast<__half2 *>(&v[i]);
+        const __half2 *gh = reinterpret_cast<const __half2 *>(&gv[i]);
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const float2 f = __half22float2(h[e2]);
+          const float2 gf = __half22float2(gh[e2]);
+          const float y0 = den > 0.f ? __fmul_rn(__fdiv_rn(f.x, den), gf.x) : 0.f;
+          const float y1 = den > 0.f ? __fmul_rn(__fdiv_rn(f.y, den), gf.y) : 0.f;
+          h[e2] = __floats2half2_rn(y0, y1);
+        }
+        if (xn_row && vi < nvec) reinterpret_cast<uint4 *>(xn_row)[vi] = v[i];
+      }
+    }
     float aI = 0.f, aN = 0.f;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
@@ -344,7 +405,7 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
 
 template <int VPT, int G, int RT>
 cudaError_t launch_variant(const QArgs &a, int grid, int cluster, cudaStream_t stream) {
-  auto kernel = quantize_act_kernel<VPT, G, RT>;
+  auto kernel = a.gamma ? quantize_act_kernel<VPT, G, RT, true> : quantize_act_kernel<VPT, G, RT, false>;
   const size_t smem = sizeof(uint32_t) * 3 * (a.K / 32);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem < 48 * 1024 ? 48 * 1024 : smem));
@@ -375,12 +436,17 @@ int quantize_max_k() { return 16 * kRowThreads * 8; }
 cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx,
                                 int K_out, float threshold, int8_t *Xq, float *s_x, void *X_out,
                                 uint32_t *bitmap, int32_t *flags, int32_t *status,
-                                cudaStream_t stream, int num_sms) {
+                                cudaStream_t stream, int num_sms, const void *gamma, float eps,
+                                void *Xn, int ldxn) {
   QArgs a{};
   a.X = static_cast<const __half *>(X);
   a.M = M;
   a.K = K;
   a.ldx = ldx;
+  a.gamma = static_cast<const __half *>(gamma);
+  a.eps = eps;
+  a.Xn = static_cast<__half *>(Xn);
+  a.ldxn = ldxn;
   a.idx = idx;
   a.K_out = K_out;
   a.K_out_pad = k_out_pad(K_out);

@@ -44,6 +44,12 @@ def weights(N: int, K: int, seed: int = SEED_W, std: float = 0.02) -> np.ndarray
     return w.astype(np.float16)
 
 
+def gains(K: int, seed: int = 11, std: float = 0.1) -> np.ndarray:
+    """fp16 [K] ~ N(1, std): the gain of an RMS normalisation before the layer."""
+    rng = np.random.default_rng(seed)
+    return (1.0 + rng.standard_normal(K, dtype=np.float32) * np.float32(std)).astype(np.float16)
+
+
 def outlier_channels(K: int, count: int, seed: int = SEED_PERM) -> np.ndarray:
     """Sorted int32 channel list: first `count` of a seeded permutation of [0, K)."""
     perm = np.random.default_rng(seed).permutation(K)

@@ -75,6 +75,24 @@ def test_host_checks_come_before_device_checks(lib):
     assert rc == 1
 
 
+def test_rmsnorm_quantize_host_checks(lib):
+    f = ctypes.c_float
+    # null gain, negative / NaN eps, short Xn stride, misaligned gain: all host errors
+    args = dict(X=0x1000, M=4, K=256, ldx=256, gamma=0x6000, eps=f(1e-5), Xn=None, ldxn=0,
+                idx=None, K_out=0, T=f(6.0), Xq=0x2000, s_x=0x3000, X_out=None, bitmap=0x4000,
+                flags=0x5000, status=None, stream=None)
+
+    def call(**kw):
+        a = dict(args, **kw)
+        return lib.mixq_rmsnorm_quantize_act(*a.values())
+
+    assert call(gamma=None) == 1
+    assert call(eps=f(-1.0)) == 1
+    assert call(eps=f(float("nan"))) == 1
+    assert call(Xn=0x7000, ldxn=128) == 1
+    assert call(gamma=0x6008) == 3
+
+
 def test_no_device_reported(lib):
     import torch
     if torch.cuda.is_available():
@@ -113,3 +131,5 @@ def test_gemm_plan_w4(lib, M, N, K):
         assert 64 <= ctas <= 2 * 148
     else:
         assert bn in (128, 256) and ctas == -(-M // 128) * -(-N // bn) * split
+        if M <= 1024:
+            assert bn == 128  # tensor-memory-operand kernel
