@@ -36,7 +36,10 @@
  *   - 4-bit level 2 uses integer scale s2 = max(1, ceil((hi-lo)/15)) and zero
  *     z2 = clamp(rint(-lo/s2), 0, 15), with q clamped so (q-z2)*s2 is int8;
  *   - the final Y is evaluated in fp64 (the kernel's fp32 epilogue is checked
- *     against it within the stated tolerance).
+ *     against it within the stated tolerance);
+ *   - the operation before the layer that the activation pass may absorb is
+ *     the Llama RMSNorm x / sqrt(mean x^2 + eps) * g, evaluated in fp64 and
+ *     rounded once to fp16 (a zero row with eps 0 stays zero).
  *
  * Floating point that decides an integer (a code, a threshold test, s2/z2) is
  * done in fp32 with single IEEE operations, the same precision the kernel
