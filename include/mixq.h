@@ -162,6 +162,32 @@ mixq_status mixq_rmsnorm_quantize_act(const void *X, int M, int K, int ldx, cons
                                       int32_t *status, void *stream);
 
 /*
+ * Outlier set kept across decode steps (MixQ article, MixQ的解决方案 Fig. 9:
+ * outliers recur in the same channels, so the set is found once and reused).
+ * When a step reports detections outside the set (flags[1] > 0), the set
+ * grows by those channels and the outlier weight columns are rebuilt; the
+ * INT8 / 4-bit codes stay as they are (the weight range covers all columns).
+ *
+ * mixq_merge_outliers (host memory only, no GPU): idx_new = sorted union of
+ * idx (sorted, unique, in [0, K)) and the channels whose bit is set in
+ * detect_bitmap [K/32] (bit k%32 of word k/32).  idx_new has room for K
+ * entries; *K_out_new receives the count.  MIXQ_ERR_INVALID_ARG for a bad K,
+ * an unsorted idx or a null pointer.
+ */
+mixq_status mixq_merge_outliers(const uint32_t *detect_bitmap, int K, const int32_t *idx,
+                                int K_out, int32_t *idx_new, int *K_out_new);
+
+/*
+ * mixq_extract_outlier_weights (device): W_out [N][K_out_pad] fp16 =
+ * W[:, idx[j]] for j < K_out in idx order, +0.0 up to K_out_pad (the W_out
+ * of mixq_prepack_weights for a new idx).  W fp16 [N][K] (the full-precision
+ * weights), idx device int32 [K_out] sorted, unique, in [0, K) (else
+ * MIXQ_ERR_INVALID_ARG in *status).  Pointers 16-byte aligned.
+ */
+mixq_status mixq_extract_outlier_weights(const void *W, int N, int K, const int32_t *idx,
+                                         int K_out, void *W_out, int32_t *status, void *stream);
+
+/*
  * Mixed-precision GEMM, 8-bit weights (MixQ Fig. 5 decomposition; Fig. 12
  * fused dequantize, scale and add of the INT32 result in registers):
  *   acc[m,n] = sum_k Xq[m,k] Wq[n,k]                     (exact INT32, tcgen05 kind::i8)

@@ -34,6 +34,8 @@ _SIGNATURES = {
     "mixq_quantize_act": (_I, [_VP, _I, _I, _I, _VP, _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
     "mixq_rmsnorm_quantize_act": (_I, [_VP, _I, _I, _I, _VP, _F, _VP, _I, _VP, _I, _F, _VP, _VP,
                                        _VP, _VP, _VP, _VP, _VP]),
+    "mixq_merge_outliers": (_I, [_VP, _I, _VP, _I, _VP, _c.POINTER(_I)]),
+    "mixq_extract_outlier_weights": (_I, [_VP, _I, _I, _VP, _I, _VP, _VP, _VP]),
     "mixq_gemm_w8a8o16": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I, _VP,
                                _VP]),
     "mixq_gemm_w4a8o16": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I,
@@ -197,6 +199,33 @@ class PackedWeights:
     @property
     def k_out(self) -> int:
         return self.idx.numel()
+
+
+def merge_outliers(bitmap, idx, K: int):
+    """Sorted union of the outlier channels idx and the channels set in a detection
+    bitmap (both device tensors), as a new device int32 tensor (host merge, one sync)."""
+    import numpy as np
+    torch = _require_cuda()
+    bm = bitmap.detach().to("cpu").contiguous().view(torch.int32).numpy().view(np.uint32)
+    old = idx.detach().to("cpu", torch.int32).contiguous().numpy()
+    out = np.empty(K, dtype=np.int32)
+    n = _I()
+    _check(lib().mixq_merge_outliers(bm.ctypes.data, K, old.ctypes.data if old.size else None,
+                                     old.size, out.ctypes.data, ctypes.byref(n)))
+    return torch.from_numpy(out[:n.value].copy()).to(idx.device if idx.numel() else bitmap.device)
+
+
+def update_outliers(w: PackedWeights, W, idx_new, status=None, stream=None) -> PackedWeights:
+    """The same prepacked codes with the outlier columns rebuilt for a new outlier set
+    (W: the layer's fp16 weights [N, K] on the device)."""
+    torch = _require_cuda()
+    idx_new = torch.as_tensor(idx_new, dtype=torch.int32, device=W.device).contiguous()
+    ko = idx_new.numel()
+    W_out = torch.empty((w.N, k_out_pad(ko)), dtype=torch.float16, device=W.device) if ko else None
+    if ko:
+        _check(lib().mixq_extract_outlier_weights(_ptr(W.contiguous()), w.N, w.K, _ptr(idx_new), ko,
+                                                  _ptr(W_out), _ptr(status), _stream(stream)))
+    return PackedWeights(w.mode, w.N, w.K, idx_new, w.Wq, w.s_w, w.grp, W_out)
 
 
 def status_tensor(device=None):

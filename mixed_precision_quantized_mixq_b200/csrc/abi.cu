@@ -138,6 +138,45 @@ mixq_status mixq_prepack_weights(int mode, const void *W, int N, int K, const in
                    "prepack launch");
 }
 
+mixq_status mixq_extract_outlier_weights(const void *W, int N, int K, const int32_t *idx,
+                                         int K_out, void *W_out, int32_t *status,
+                                         void *stream) {
+  mixq_status s = check_shape(0, N, K, K_out);
+  if (s != MIXQ_OK) return s;
+  if (K_out == 0) return ok();
+  if (!W || !idx || !W_out) return fail(MIXQ_ERR_INVALID_ARG, "W, idx and W_out must be non-null");
+  if (!aligned16(W) || !aligned16(W_out))
+    return fail(MIXQ_ERR_MISALIGNED, "W and W_out must be 16-byte aligned");
+  s = check_device(nullptr);
+  if (s != MIXQ_OK) return s;
+  return from_cuda(mixq::launch_extract_outliers(W, N, K, idx, K_out, W_out, status,
+                                                 static_cast<cudaStream_t>(stream)),
+                   "outlier extraction launch");
+}
+
+mixq_status mixq_merge_outliers(const uint32_t *detect_bitmap, int K, const int32_t *idx,
+                                int K_out, int32_t *idx_new, int *K_out_new) {
+  if (K <= 0 || K % 32 || K_out < 0 || K_out > K || !detect_bitmap || !idx_new || !K_out_new ||
+      (K_out > 0 && !idx))
+    return fail(MIXQ_ERR_INVALID_ARG, "merge: bad K, K_out or null pointer");
+  // sorted union of idx and the detected channels: one pass over the channels
+  int j = 0, n = 0;
+  for (int c = 0; c < K; ++c) {
+    bool in_idx = false;
+    if (j < K_out && idx[j] == c) {
+      in_idx = true;
+      ++j;
+    } else if (j < K_out && (idx[j] < c || idx[j] >= K || (j > 0 && idx[j] <= idx[j - 1]))) {
+      return fail(MIXQ_ERR_INVALID_ARG, "merge: idx must be sorted, unique, inside [0, K)");
+    }
+    const bool detected = (detect_bitmap[c >> 5] >> (c & 31)) & 1u;
+    if (in_idx || detected) idx_new[n++] = c;
+  }
+  if (j != K_out) return fail(MIXQ_ERR_INVALID_ARG, "merge: idx must be sorted, unique, inside [0, K)");
+  *K_out_new = n;
+  return ok();
+}
+
 static mixq_status quantize_common(const void *X, int M, int K, int ldx, const int32_t *idx,
                                    int K_out, float threshold, int8_t *Xq, float *s_x,
                                    void *X_out, uint32_t *detect_bitmap, int32_t *flags,

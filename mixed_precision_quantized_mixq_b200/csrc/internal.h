@@ -30,6 +30,8 @@ cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int3
 cudaError_t launch_prepack(int mode, const void *W, int N, int K, const int32_t *idx, int K_out,
                            void *Wq, float *s_w, void *grp, void *W_out, int32_t *status,
                            cudaStream_t stream);
+cudaError_t launch_extract_outliers(const void *W, int N, int K, const int32_t *idx, int K_out,
+                                    void *W_out, int32_t *status, cudaStream_t stream);
 cudaError_t launch_unpack_w8(int N, int K, const void *Wq, int8_t *out, cudaStream_t stream);
 cudaError_t launch_unpack_w4(int N, int K, const void *Wq4, const void *grp, uint8_t *q,
                              uint8_t *s2, uint8_t *z2, cudaStream_t stream);

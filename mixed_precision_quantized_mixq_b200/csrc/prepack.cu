@@ -203,6 +203,28 @@ __global__ void unpack_w4_kernel(int N, int K, const uint8_t *__restrict__ Wq4,
   }
 }
 
+// Outlier weight columns alone, in idx order (MixQ Fig. 11), for an outlier
+// set that changed after the prepack: W_out[n][j] = W[n][idx[j]] for j < K_out,
+// +0.0 up to K_out_pad.  The INT8/4-bit codes do not depend on idx (the weight
+// range covers every column), so only these columns are rebuilt.
+__global__ void __launch_bounds__(256) extract_outlier_kernel(
+    const __half *__restrict__ W, int N, int K, const int32_t *__restrict__ idx, int K_out,
+    int K_out_pad, __half *__restrict__ W_out, int32_t *__restrict__ status) {
+  for (int n = blockIdx.x; n < N; n += gridDim.x) {
+    const __half *wh = W + static_cast<size_t>(n) * K;
+    for (int j = threadIdx.x; j < K_out_pad; j += blockDim.x) {
+      __half v = __ushort_as_half(0);
+      if (j < K_out) {
+        const int c = idx[j];
+        const bool ok = c >= 0 && c < K && (j == 0 || idx[j - 1] < c);
+        if (ok) v = wh[c];
+        else record_error(status, kErrInvalidArg);
+      }
+      W_out[static_cast<size_t>(n) * K_out_pad + j] = v;
+    }
+  }
+}
+
 __global__ void unpack_w8_kernel(int N, int K, const int8_t *__restrict__ Wq,
                                  int8_t *__restrict__ out) {
   const size_t total = static_cast<size_t>(N) * K;
@@ -234,6 +256,17 @@ cudaError_t launch_prepack(int mode, const void *W, int N, int K, const int32_t 
         static_cast<const __half *>(W), N, K, idx, K_out, k_out_pad(K_out), Wq, s_w,
         static_cast<__half2 *>(grp), static_cast<__half *>(W_out), status);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_extract_outliers(const void *W, int N, int K, const int32_t *idx, int K_out,
+                                    void *W_out, int32_t *status, cudaStream_t stream) {
+  const int kp = k_out_pad(K_out);
+  if (N == 0 || kp == 0) return cudaSuccess;
+  const int grid = N < 8192 ? N : 8192;
+  extract_outlier_kernel<<<grid, 256, 0, stream>>>(static_cast<const __half *>(W), N, K, idx,
+                                                   K_out, kp, static_cast<__half *>(W_out),
+                                                   status);
   return cudaGetLastError();
 }
 

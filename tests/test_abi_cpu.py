@@ -2,6 +2,8 @@
 include/mixq.h declares, and does its host-side work (argument checks, size
 queries, launch planning) without touching a device."""
 import ctypes
+
+import numpy as np
 import os
 import re
 
@@ -91,6 +93,45 @@ def test_rmsnorm_quantize_host_checks(lib):
     assert call(eps=f(float("nan"))) == 1
     assert call(Xn=0x7000, ldxn=128) == 1
     assert call(gamma=0x6008) == 3
+
+
+def _merge(lib, bitmap, idx, K):
+    bitmap = np.ascontiguousarray(bitmap, np.uint32)
+    idx = np.ascontiguousarray(idx, np.int32)
+    out = np.full(K, -1, np.int32)
+    n = ctypes.c_int(-1)
+    rc = lib.mixq_merge_outliers(bitmap.ctypes.data, K, idx.ctypes.data if idx.size else None,
+                                 idx.size, out.ctypes.data, ctypes.byref(n))
+    return rc, out[:max(n.value, 0)]
+
+
+def test_merge_outliers_is_the_sorted_union(lib):
+    # host-only call: the outlier set grows by the channels detected outside it
+    rng = np.random.default_rng(3)
+    for K in (32, 256, 4096):
+        for _ in range(20):
+            idx = np.sort(rng.choice(K, rng.integers(0, K // 4 + 1), replace=False)).astype(np.int32)
+            det = rng.choice(K, rng.integers(0, K // 8 + 1), replace=False)
+            bitmap = np.zeros(K // 32, np.uint32)
+            for c in det:
+                bitmap[c // 32] |= np.uint32(1) << np.uint32(c % 32)
+            rc, got = _merge(lib, bitmap, idx, K)
+            assert rc == 0
+            np.testing.assert_array_equal(got, np.union1d(idx, det).astype(np.int32))
+    # all channels detected -> every channel; nothing detected -> idx unchanged
+    rc, got = _merge(lib, np.full(8, 0xFFFFFFFF, np.uint32), np.array([5, 9], np.int32), 256)
+    assert rc == 0 and np.array_equal(got, np.arange(256))
+    rc, got = _merge(lib, np.zeros(8, np.uint32), np.array([5, 9], np.int32), 256)
+    assert rc == 0 and np.array_equal(got, [5, 9])
+
+
+def test_merge_outliers_rejects_bad_input(lib):
+    z = np.zeros(8, np.uint32)
+    assert _merge(lib, z, np.array([9, 5], np.int32), 256)[0] == 1      # unsorted
+    assert _merge(lib, z, np.array([5, 5], np.int32), 256)[0] == 1      # duplicate
+    assert _merge(lib, z, np.array([-1], np.int32), 256)[0] == 1        # out of range
+    assert _merge(lib, z, np.array([300], np.int32), 256)[0] == 1       # out of range
+    assert _merge(lib, np.zeros(1, np.uint32), np.array([], np.int32), 33)[0] == 1  # K % 32
 
 
 def test_no_device_reported(lib):
