@@ -221,11 +221,10 @@ mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
 
 /*
  * The launch plan the gemm calls use for a shape (host only, no GPU needed):
- * output tile width *bn in output channels (MIXQ_W8, and MIXQ_W4G128 above
- * M = 1024: 128 or 256, tiles 128 tokens high; MIXQ_W4G128 up to M = 1024:
- * 128, tiles of up to 128 tokens, all tokens when M <= 64), the K-split
- * factor *split (thread-block cluster size along K, 1..8) and the number of
- * CTAs *ctas.  num_sms <= 0 means "query the current device" (and, for the
+ * output tile width *bn in output channels (MIXQ_W8: 32, 64, 128 or 256,
+ * tiles 128 tokens high; MIXQ_W4G128: 128, tiles of all tokens when M <= 64,
+ * 128 tokens up to M = 1024, 256 tokens above), the K-split factor *split
+ * (thread-block cluster size along K, 1..8) and the number of CTAs *ctas.  num_sms <= 0 means "query the current device" (and, for the
  * shared-memory-operand kernel, its cluster occupancy).  That kernel with
  * bn <= 128 runs the variant that fits two CTAs per SM (token-sized A slots
  * when M <= 64).
@@ -240,9 +239,9 @@ mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, 
  * 64 need M <= 64; with M <= 64 and bn <= 128 the small-M variant runs.
  * MIXQ_W4G128: bn 128 = the tensor-memory-operand kernel's two-CTA-per-SM
  * variant (a K split only with M <= 64, else MIXQ_ERR_UNSUPPORTED_SHAPE),
- * 256 = its one-CTA-per-SM variant, 32/64 = the shared-memory-operand
- * kernel with narrow tiles (M <= 64); 0 = the plan (tensor-memory operand up
- * to M = 1024, shared-memory operand above).
+ * 256 = its one-CTA-per-SM variant (256-token tiles above M = 1024, where it
+ * splits no K), 32/64 = the shared-memory-operand
+ * kernel with narrow tiles (M <= 64); 0 = the plan.
  */
 mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq, const void *Wq,
                                 const void *grp, int32_t *acc, int ldacc, int bn, int split,

@@ -269,9 +269,9 @@ static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const i
   a.epi = mixq::Epi::kMixed;
   a.status = status;
   a.wait_limit_ns = kDefaultWaitNs;
-  // (the W4 planner below M = 1024 needs no occupancy table)
+  // (the W4 planner needs no occupancy table)
   const mixq::GemmPlan plan = mixq::plan_gemm(
-      mode, M, N, K, sms, (mode == MIXQ_W8 || M > 1024) ? mixq::device_cluster_limits(mode) : nullptr);
+      mode, M, N, K, sms, mode == MIXQ_W8 ? mixq::device_cluster_limits(mode) : nullptr);
   const char *why = nullptr;
   const cudaError_t e = mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why);
   return from_cuda(e, "gemm launch", why);
@@ -341,6 +341,9 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   if (mode == MIXQ_W4G128 && bn == 128 && split > 1 && M > 64)
     return fail(MIXQ_ERR_UNSUPPORTED_SHAPE,
                 "W4 two-CTA variant (bn = 128) splits K only for M <= 64");
+  if (mode == MIXQ_W4G128 && bn == 256 && split > 1 && M > 1024)
+    return fail(MIXQ_ERR_UNSUPPORTED_SHAPE,
+                "W4 one-CTA variant (bn = 256) splits K only for M <= 1024");
   if (M == 0) return check_device(nullptr);
   if (!Xq || !Wq || !acc || (mode == MIXQ_W4G128 && !grp))
     return fail(MIXQ_ERR_INVALID_ARG, "null pointer");
@@ -350,7 +353,7 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   s = check_device(&sms);
   if (s != MIXQ_OK) return s;
   mixq::GemmPlan plan = mixq::plan_gemm(
-      mode, M, N, K, sms, (mode == MIXQ_W8 || M > 1024) ? mixq::device_cluster_limits(mode) : nullptr);
+      mode, M, N, K, sms, mode == MIXQ_W8 ? mixq::device_cluster_limits(mode) : nullptr);
   if (split) plan.split = split;
   if (mode == MIXQ_W4G128 && (bn == 128 || bn == 256 || (bn == 0 && plan.ts))) {
     // tensor-memory-operand kernel: bn = 128 the two-CTA-per-SM variant,

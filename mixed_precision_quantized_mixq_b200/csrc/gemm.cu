@@ -803,11 +803,12 @@ int decode_split(int n_tiles, int KB, int num_sms) {
 }
 
 GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimits *limits) {
-  // W4 up to M = 1024: expanded weights in tensor memory (measured against
-  // the smem operand on the Llama shapes: 1.4x at M = 16, 1.13x at M = 512,
-  // up to 1.24x at M = 512 with N = 28672; within +-4% at M = 2048 and 8192,
-  // where the smem x smem kernel below keeps W4)
-  if (mode == 1 && M <= 1024) return plan_gemm_w4ts(M, N, K, num_sms);
+  // W4: expanded weights in tensor memory at every M (measured against the
+  // smem operand on the Llama shapes: 1.4x at M = 16, 1.13x at M = 512, up to
+  // 1.24x at M = 512 with N = 28672, 0-5 % at M = 2048 and 8192 with 256-token
+  // tiles).  The W4 branches of the smem x smem kernel remain for the
+  // narrow-tile debug launches.
+  if (mode == 1) return plan_gemm_w4ts(M, N, K, num_sms);
   if (M <= 64) {
     (void)limits;
     const int split = decode_split(N / 128, K / kBlockK, num_sms);

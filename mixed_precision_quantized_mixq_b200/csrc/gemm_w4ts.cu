@@ -64,7 +64,7 @@ constexpr int kTsPacked = 128 * (kBlockK / 2);        // 8 KB of codes per 128 x
 constexpr int kTsGrp = 128 * 4;                        // (s2, z2) fp16 pair per row
 constexpr int kTsOutK = 32;                            // fp16 K per outlier stage (64 bytes)
 constexpr int kTsWOut = 128 * kTsOutK * 2;             // W_out tile of an outlier stage
-constexpr int kTsExtra = 1024 + 512 + 512;             // barriers, s_w[128], s_x[128]
+constexpr int kTsExtra = 1024 + 512 + 1024;            // barriers, s_w[128], s_x[256]
 constexpr int kTsPitch = 128 + 4;                      // words per token row of a partial tile
 
 // SM = two CTAs per SM (half the shared memory, 256 TMEM columns each): the
@@ -86,7 +86,7 @@ struct TsCfg {
 // holds a 32-column W_out tile at 0 and the X_out tile at w_slot.
 struct TsParams {
   int M, N, K, K_out_pad;
-  int bt;           // tokens per tile = MMA N (multiple of 16, at most 128)
+  int bt;           // tokens per tile = MMA N (multiple of 16, at most 256)
   int kbpj;         // K blocks per job (1 or 2)
   int stages;       // shared-memory ring depth (>= a_stages)
   int stage_bytes;  // w_slot + kbpj * bt * 128
@@ -194,7 +194,7 @@ __global__ void __launch_bounds__(kTsThreads, TsCfg<SM>::kMinBlocks)
   uint32_t *tmem_holder = reinterpret_cast<uint32_t *>(i8_done + 1);
   int *s_misc = reinterpret_cast<int *>(tmem_holder + 1);  // err, weights issued, tokens issued
   float *s_sw = reinterpret_cast<float *>(extra + 1024);   // [128]
-  float *s_sx = reinterpret_cast<float *>(extra + 1536);   // [bt]
+  float *s_sx = reinterpret_cast<float *>(extra + 1536);   // [bt], bt <= 256
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bt = p.bt;
@@ -602,7 +602,9 @@ template <bool SM>
 TsGeometry ts_geometry(int M) {
   using C = TsCfg<SM>;
   TsGeometry g{};
-  g.bt = SM ? (M >= 128 ? 128 : (M + 15) / 16 * 16) : 128;
+  // the one-CTA variant takes 256 tokens per tile above M = 1024 (MMA N = 256:
+  // half the token-tile bytes per MAC of a 128-token tile)
+  g.bt = SM ? (M >= 128 ? 128 : (M + 15) / 16 * 16) : (M > 1024 ? 256 : 128);
   if (g.bt < 16) g.bt = 16;
   // two K blocks per job unless that leaves fewer than three stages
   for (int kbpj = 2; kbpj >= 1; --kbpj) {
@@ -614,6 +616,7 @@ TsGeometry ts_geometry(int M) {
     if (g.stages >= 3) break;
   }
   g.a_stages = (C::kTmemCols - C::kACol) / (32 * g.kbpj);
+  if (g.a_stages > g.stages) g.a_stages = g.stages;
   g.smem = g.stages * g.stage_bytes + kTsExtra + 1024;
   g.f32_col = 2 * g.bt <= C::kACol ? g.bt : C::kACol;
   return g;
@@ -706,6 +709,12 @@ GemmPlan plan_gemm_w4ts(int M, int N, int K, int num_sms) {
   if (M <= 64) {
     const int split = decode_split(n_tiles, KB, num_sms);
     return GemmPlan{128, split, n_tiles * split, 1, 1};
+  }
+  if (M > 1024) {
+    // one CTA per SM with 256-token tiles: half the token-tile bytes per MAC of
+    // a 128-token tile (measured 0-5 % ahead of the two-CTA 128-token variant
+    // and of the smem-operand kernel at M = 2048 and 8192)
+    return GemmPlan{128, 1, (M + 255) / 256 * n_tiles, 0, 1};
   }
   const int m_tiles = (M + 127) / 128;
   const int ctas = m_tiles * n_tiles;

@@ -76,9 +76,9 @@ struct GemmArgs {
   int debug_stall;  // producer issues nothing (timeout test)
 };
 
-// W8, and W4 at M > 1024, run the smem x smem kernel (gemm.cu); W4 at
-// M <= 1024 runs the kernel that keeps the expanded weights in tensor memory
-// (gemm_w4ts.cu, plan.ts = 1).
+// W8 runs the smem x smem kernel (gemm.cu); W4 runs the kernel that keeps the
+// expanded weights in tensor memory (gemm_w4ts.cu, plan.ts = 1), except the
+// narrow-tile debug launches.
 cudaError_t launch_gemm(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
                         const char **why);
 GemmPlan plan_gemm_w4ts(int M, int N, int K, int num_sms);

@@ -170,7 +170,9 @@ def test_gemm_plan_w4(lib, M, N, K):
         # tensor-memory-operand kernel: 128 weight rows x all tokens per tile
         assert bn == 128 and ctas == (N // 128) * split
         assert 64 <= ctas <= 2 * 148
+    elif M <= 1024:
+        # tensor-memory-operand kernel, 128-token tiles
+        assert bn == 128 and ctas == -(-M // 128) * (N // 128) * split
     else:
-        assert bn in (128, 256) and ctas == -(-M // 128) * -(-N // bn) * split
-        if M <= 1024:
-            assert bn == 128  # tensor-memory-operand kernel
+        # one CTA per SM, 256-token tiles, no K split
+        assert bn == 128 and split == 1 and ctas == -(-M // 256) * (N // 128)
