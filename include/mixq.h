@@ -221,13 +221,13 @@ mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
 
 /*
  * The launch plan the gemm calls use for a shape (host only, no GPU needed):
- * output tile width *bn in output channels (MIXQ_W8: 32, 64, 128 or 256,
- * tiles 128 tokens high; MIXQ_W4G128: 128, tiles of all tokens when M <= 64,
- * 128 tokens up to M = 1024, 256 tokens above), the K-split factor *split
- * (thread-block cluster size along K, 1..8) and the number of CTAs *ctas.  num_sms <= 0 means "query the current device" (and, for the
- * shared-memory-operand kernel, its cluster occupancy).  That kernel with
- * bn <= 128 runs the variant that fits two CTAs per SM (token-sized A slots
- * when M <= 64).
+ * output tile width *bn in output channels (always 128: MIXQ_W8 tiles are
+ * 128 tokens high, two CTAs per SM, token-sized A slots when M <= 64;
+ * MIXQ_W4G128 tiles hold all tokens when M <= 64, 128 tokens up to M = 1024,
+ * 256 tokens above), the K-split factor *split (thread-block cluster size
+ * along K, 1..8; used at M <= 64, and for W4 tiles too few to fill the SMs)
+ * and the number of CTAs *ctas.  num_sms <= 0 means "query the current
+ * device".
  */
 mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, int *split,
                            int *ctas);

@@ -269,9 +269,7 @@ static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const i
   a.epi = mixq::Epi::kMixed;
   a.status = status;
   a.wait_limit_ns = kDefaultWaitNs;
-  // (the W4 planner needs no occupancy table)
-  const mixq::GemmPlan plan = mixq::plan_gemm(
-      mode, M, N, K, sms, mode == MIXQ_W8 ? mixq::device_cluster_limits(mode) : nullptr);
+  const mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms);
   const char *why = nullptr;
   const cudaError_t e = mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why);
   return from_cuda(e, "gemm launch", why);
@@ -298,13 +296,11 @@ mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, 
   if (mode != MIXQ_W8 && mode != MIXQ_W4G128) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
   mixq_status s = check_shape(M, N, K, 0);
   if (s != MIXQ_OK) return s;
-  const mixq::ClusterLimits *limits = nullptr;
   if (num_sms <= 0) {
     s = check_device(&num_sms);
     if (s != MIXQ_OK) return s;
-    limits = mixq::device_cluster_limits(mode);
   }
-  const mixq::GemmPlan p = mixq::plan_gemm(mode, M, N, K, num_sms, limits);
+  const mixq::GemmPlan p = mixq::plan_gemm(mode, M, N, K, num_sms);
   if (bn) *bn = p.bn;
   if (split) *split = p.split;
   if (ctas) *ctas = p.ctas;
@@ -352,8 +348,7 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   int sms = 0;
   s = check_device(&sms);
   if (s != MIXQ_OK) return s;
-  mixq::GemmPlan plan = mixq::plan_gemm(
-      mode, M, N, K, sms, mode == MIXQ_W8 ? mixq::device_cluster_limits(mode) : nullptr);
+  mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms);
   if (split) plan.split = split;
   if (mode == MIXQ_W4G128 && (bn == 128 || bn == 256 || (bn == 0 && plan.ts))) {
     // tensor-memory-operand kernel: bn = 128 the two-CTA-per-SM variant,
@@ -438,7 +433,7 @@ mixq_status mixq_debug_gemm_stall(int M, int N, int K, const int8_t *Xq, const v
   a.status = status;
   a.wait_limit_ns = wait_limit_ns;
   a.debug_stall = 1;
-  mixq::GemmPlan plan = mixq::plan_gemm(MIXQ_W8, M, N, K, sms, nullptr);
+  mixq::GemmPlan plan = mixq::plan_gemm(MIXQ_W8, M, N, K, sms);
   plan.split = 1;
   plan.bn = 128;
   plan.small_m = M <= 64 ? 1 : 0;

@@ -739,28 +739,6 @@ int max_active_clusters_variant(int split) {
 
 }  // namespace
 
-const ClusterLimits *device_cluster_limits(int mode) {
-  static ClusterLimits table[64][2];
-  static std::atomic<int> ready[64][2];
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
-  const int md = mode == 1 ? 1 : 0;
-  if (ready[dev][md].load(std::memory_order_acquire)) return &table[dev][md];
-  static std::mutex mu;
-  std::lock_guard<std::mutex> lock(mu);
-  if (!ready[dev][md].load(std::memory_order_acquire)) {
-    ClusterLimits &t = table[dev][md];
-    for (int small = 0; small < 2; ++small)
-      for (int wide = 0; wide < 2; ++wide)
-        for (int s = 0; s <= 8; ++s)
-          t.max_active[small][wide][s] =
-              (s == 0 || (small && wide)) ? 0
-                                          : gemm_max_active_clusters(md, wide ? 256 : 128, s, small);
-    ready[dev][md].store(1, std::memory_order_release);
-  }
-  return &table[dev][md];
-}
-
 int gemm_max_active_clusters(int mode, int bn, int split, int small_m) {
   if (small_m) {
     if (bn == 32) return mode == 1 ? max_active_clusters_variant<32, true, true>(split)
@@ -775,13 +753,6 @@ int gemm_max_active_clusters(int mode, int bn, int split, int small_m) {
                                   : max_active_clusters_variant<256, false, false>(split);
   return mode == 1 ? max_active_clusters_variant<128, true, false>(split)
                    : max_active_clusters_variant<128, false, false>(split);
-}
-
-int estimate_max_active_clusters(int num_sms, int ctas_per_sm, int split) {
-  // SMs come in GPCs of about 18 and a cluster lives inside one GPC.
-  const int gpcs = (num_sms + 9) / 18 > 0 ? (num_sms + 9) / 18 : 1;
-  const int per_gpc = num_sms / gpcs;
-  return gpcs * ((per_gpc * ctas_per_sm) / split);
 }
 
 int decode_split(int n_tiles, int KB, int num_sms) {
@@ -802,80 +773,23 @@ int decode_split(int n_tiles, int KB, int num_sms) {
   return best;
 }
 
-GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimits *limits) {
+GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms) {
   // W4: expanded weights in tensor memory at every M (measured against the
   // smem operand on the Llama shapes: 1.4x at M = 16, 1.13x at M = 512, up to
   // 1.24x at M = 512 with N = 28672, 0-5 % at M = 2048 and 8192 with 256-token
   // tiles).  The W4 branches of the smem x smem kernel remain for the
   // narrow-tile debug launches.
   if (mode == 1) return plan_gemm_w4ts(M, N, K, num_sms);
+  const int n128 = (N + 127) / 128;
   if (M <= 64) {
-    (void)limits;
-    const int split = decode_split(N / 128, K / kBlockK, num_sms);
-    return GemmPlan{128, split, N / 128 * split, 1};
+    const int split = decode_split(n128, K / kBlockK, num_sms);
+    return GemmPlan{128, split, n128 * split, 1};
   }
-  // Time model (microseconds at ~1.9 GHz).  CTAs run in waves; a wave holds
-  // at most max_active(split) clusters of `split` CTAs (one CTA per SM; two for
-  // the small-M variants).  A K block costs a CTA the larger of its MMA cycles
-  // (8192 INT8 MACs per cycle) and its shared-memory cycles (the MMA reads all
-  // 128 A rows plus the BN B rows at 128 B per cycle) -- narrow tiles are
-  // shared-memory bound.  Fixed cost per CTA: prologue/epilogue, plus the
-  // cluster reduction (which waits for the slowest peer) when K is split.
-  // Memory: the bytes that must come from HBM at least once (weights,
-  // activations, output) at the HBM rate.  Cost = max(compute, memory); ties
-  // keep fewer CTAs.
-  const int m_tiles = (M + kTileM - 1) / kTileM;
-  {
-    // Prefill-sized M.  W8: two 128 x 128 CTAs per SM (about 100 KB each), so
-    // one CTA's epilogue overlaps the other's mainloop and the grid packs
-    // into waves twice as finely (measured better than one 128 x 256 CTA per
-    // SM on every workload shape).  W4: its expansion needs the deeper
-    // one-CTA-per-SM pipeline, unless that grid wastes more than 15% of its
-    // last wave.
-    const int n128 = (N + 127) / 128;
-    if (mode != 1) return GemmPlan{128, 1, m_tiles * n128, 1};
-    const long long ctas256 = static_cast<long long>(m_tiles) * ((N + 255) / 256);
-    const double waves = static_cast<double>(ctas256) / num_sms;
-    const double tail_eff = waves / static_cast<double>((ctas256 + num_sms - 1) / num_sms);
-    if (tail_eff < 0.85) return GemmPlan{128, 1, m_tiles * n128, 1};
-  }
-  GemmPlan best{256, 1, 0, 0};
-  double best_cost = 1e300;
-  const int KB = K / kBlockK;
-  const double w_bytes = (mode == 1 ? 0.5 + 4.0 / kGroup : 1.0) * static_cast<double>(N) * K;
-  const double unique_bytes = w_bytes + static_cast<double>(M) * K + 2.0 * M * N;
-  struct Variant { int bn, small; };
-  const Variant variants[2] = {{256, 0}, {128, 0}};
-  for (const Variant v : variants) {
-    const int wide = v.bn == 256 ? 1 : 0;
-    const double mma_cyc = 4.0 * 128 * v.bn * 32 / 8192.0;
-    const double smem_cyc = (16384.0 + v.bn * 128.0) / 128.0;
-    const double t_kb = (mma_cyc > smem_cyc ? mma_cyc : smem_cyc) / 1900.0;
-    const int n_tiles = (N + v.bn - 1) / v.bn;
-    for (int s = 1; s <= 8 && s <= KB; ++s) {
-      int clusters_per_wave = 0;
-      if (limits && v.bn >= 128)
-        clusters_per_wave = limits->max_active[v.small][wide][s];
-      else if (limits && limits->max_active[1][0][s] > 0)
-        clusters_per_wave = limits->max_active[1][0][s];  // narrow tiles: same footprint class
-      else
-        clusters_per_wave = estimate_max_active_clusters(num_sms, v.small ? 2 : 1, s);
-      if (clusters_per_wave <= 0) continue;
-      const long long slots = static_cast<long long>(clusters_per_wave) * s;
-      const long long ctas = static_cast<long long>(m_tiles) * n_tiles * s;
-      const long long waves = (ctas + slots - 1) / slots;
-      const int kb_per = (KB + s - 1) / s;
-      const double fixed = 1.5 + (s > 1 ? 1.5 + 0.05 * s : 0.0);
-      const double compute = waves * (kb_per * t_kb + fixed);
-      const double memory = unique_bytes / 6.5e6 + fixed;
-      const double cost = compute > memory ? compute : memory;
-      if (cost < best_cost * (1 - 1e-6)) {
-        best_cost = cost;
-        best = GemmPlan{v.bn, s, static_cast<int>(ctas), v.small};
-      }
-    }
-  }
-  return best;
+  // Prefill-sized M: two 128 x 128 CTAs per SM (about 100 KB each), so one
+  // CTA's epilogue overlaps the other's mainloop and the grid packs into waves
+  // twice as finely (measured better than one 128 x 256 CTA per SM, with or
+  // without a K split, on every workload shape).
+  return GemmPlan{128, 1, (M + kTileM - 1) / kTileM * n128, 1};
 }
 
 cudaError_t launch_gemm(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,

@@ -45,15 +45,10 @@ struct GemmPlan {
   int ts;       // W4 through the tensor-memory-operand kernel (gemm_w4ts.cu)
 };
 
-// How many clusters of `split` CTAs run at once, per [small-M][bn == 256][split].
-struct ClusterLimits {
-  int max_active[2][2][9];
-};
-// limits == nullptr: estimate from num_sms (GPCs of about 18 SMs).
-GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms, const ClusterLimits *limits);
-int estimate_max_active_clusters(int num_sms, int ctas_per_sm, int split);
-int gemm_max_active_clusters(int mode, int bn, int split, int small_m);  // -1 on error
-const ClusterLimits *device_cluster_limits(int mode);  // current device, cached; may be null
+GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms);
+// Clusters of `split` CTAs of the smem x smem kernel the current device runs at
+// once (-1 on error); a diagnostic for the debug entry point.
+int gemm_max_active_clusters(int mode, int bn, int split, int small_m);
 
 enum class Epi { kMixed = 0, kRawI32 = 1 };
 
