@@ -122,14 +122,38 @@ def quantize_launches(M: int, K: int) -> int:
     return 2
 
 
+def _code_only(text: str) -> str:
+    """C/C++ source without its comments and blank lines (string literals kept)."""
+    out, i, n = [], 0, len(text)
+    while i < n:
+        c = text[i]
+        if c == '"':  # string literal: copy through the closing quote
+            j = i + 1
+            while j < n and text[j] != '"':
+                j += 2 if text[j] == "\\" else 1
+            out.append(text[i:j + 1])
+            i = j + 1
+        elif text.startswith("//", i):
+            i = text.find("\n", i)
+            i = n if i < 0 else i
+        elif text.startswith("/*", i):
+            j = text.find("*/", i + 2)
+            i = n if j < 0 else j + 2
+        else:
+            out.append(c)
+            i += 1
+    return "\n".join(ln.rstrip() for ln in "".join(out).splitlines() if ln.strip())
+
+
 def kernel_source_hash() -> str:
-    """Hash of every kernel source file: committed ncu counters apply only to these sources."""
+    """Hash of the code (comments stripped) of every kernel source file: committed ncu
+    counters apply only to this code."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixed_precision_quantized_mixq_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
         if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), "rb") as fh:
-                h.update(f.encode() + b"\0" + fh.read())
+            with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+                h.update(f.encode() + b"\0" + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 

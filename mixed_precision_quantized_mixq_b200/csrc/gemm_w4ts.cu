@@ -603,7 +603,7 @@ TsGeometry ts_geometry(int M) {
   using C = TsCfg<SM>;
   TsGeometry g{};
   // the one-CTA variant takes 256 tokens per tile above M = 1024 (MMA N = 256:
-  // half the token-tile bytes per MAC of a 128-token tile)
+  // each 8.5 KB stage of codes feeds twice the tokens of a 128-token tile)
   g.bt = SM ? (M >= 128 ? 128 : (M + 15) / 16 * 16) : (M > 1024 ? 256 : 128);
   if (g.bt < 16) g.bt = 16;
   // two K blocks per job unless that leaves fewer than three stages
@@ -711,8 +711,8 @@ GemmPlan plan_gemm_w4ts(int M, int N, int K, int num_sms) {
     return GemmPlan{128, split, n_tiles * split, 1, 1};
   }
   if (M > 1024) {
-    // one CTA per SM with 256-token tiles: half the token-tile bytes per MAC of
-    // a 128-token tile (measured 0-5 % ahead of the two-CTA 128-token variant
+    // one CTA per SM with 256-token tiles: half the code bytes per MAC of a
+    // 128-token tile (measured 0-5 % ahead of the two-CTA 128-token variant
     // and of the smem-operand kernel at M = 2048 and 8192)
     return GemmPlan{128, 1, (M + 255) / 256 * n_tiles, 0, 1};
   }
