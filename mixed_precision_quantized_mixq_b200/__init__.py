@@ -228,6 +228,33 @@ def update_outliers(w: PackedWeights, W, idx_new, status=None, stream=None) -> P
     return PackedWeights(w.mode, w.N, w.K, idx_new, w.Wq, w.s_w, w.grp, W_out)
 
 
+def column_shard(N: int, rank: int, world: int) -> tuple[int, int]:
+    """Output channels [n0, n1) that one rank holds in an N-split (column-parallel)
+    layer: equal shards of whole 128-channel weight tiles."""
+    if world < 1 or not 0 <= rank < world or N % (128 * world):
+        raise ValueError(f"N = {N} does not split into {world} shards of whole 128-channel tiles")
+    per = N // world
+    return rank * per, (rank + 1) * per
+
+
+def prepack_shard(W, idx, mode: int, rank: int, world: int, status=None,
+                  stream=None) -> PackedWeights:
+    """Prepack this rank's rows of W [N, K] for an N-split layer (each output channel
+    is quantized on its own, so a shard's codes equal those rows of the full prepack)."""
+    n0, n1 = column_shard(W.shape[0], rank, world)
+    return prepack(W[n0:n1], idx, mode, status=status, stream=stream)
+
+
+def gather_columns(Y_local, world: int, group=None):
+    """All-gather the [M, N/world] output shards of an N-split layer into [M, N] in rank
+    order, over torch.distributed (NCCL between GPUs)."""
+    import torch
+    import torch.distributed as dist
+    parts = [torch.empty_like(Y_local) for _ in range(world)]
+    dist.all_gather(parts, Y_local.contiguous(), group=group)
+    return torch.cat(parts, dim=1)
+
+
 def status_tensor(device=None):
     torch = _require_cuda()
     return torch.zeros(1, dtype=torch.int32, device=device or "cuda")
