@@ -25,7 +25,7 @@
  *            asymmetric group-wise weights, two-stage dequantization on INT8
  *            tensor cores).
  *
- * Readings where the pages are silent (each one is listed in the design doc):
+ * Readings where the pages are silent (the same list is kept in the design notes):
  *   - scales are fp32; codes are symmetric in [-127, 127]; rounding is
  *     round-half-to-even of one fp32 multiply by the fp32 reciprocal 127/a;
  *   - the weight range a = max |W[n,:]| runs over ALL K columns;
