@@ -166,7 +166,8 @@ def test_int32_accumulators_bit_exact(gpu, mode, M, N, K, bn, split):
 @pytest.mark.parametrize("mode", ["w8", "w4"])
 @pytest.mark.parametrize("M,K,N,k_out", [(16, 512, 256, 4), (64, 1024, 640, 64), (130, 512, 384, 1),
                                          (260, 768, 512, 130), (8, 1024, 1024, 0),
-                                         (1, 2048, 512, 64)])
+                                         (1, 2048, 512, 64), (24, 1024, 512, 16),
+                                         (40, 2048, 384, 32)])
 def test_layer_output_within_tolerance(gpu, mode, M, K, N, k_out):
     idx = synth.outlier_channels(K, k_out)
     X = synth.activations(M, K, idx, synth.channel_factors(k_out)) if k_out else \
