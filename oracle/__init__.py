@@ -105,6 +105,43 @@ def prepack_w4(Wq8: np.ndarray):
     return q, s2, z2, w8
 
 
+def prepack_w4b(W: np.ndarray):
+    """4-bit reading B: per (row, group of 128) fp16 scale and integer zero.
+
+    Returns logical (q u8 [N,K], s_g f16 [N,K/128], z_g u8 [N,K/128])."""
+    lib = _load()
+    N, K = W.shape
+    q = np.empty((N, K), np.uint8)
+    s_g = np.empty((N, K // GROUP), np.uint16)
+    z_g = np.empty((N, K // GROUP), np.uint8)
+    rc = lib.oracle_prepack_w4b(_p(_f16bits(W)), N, K, _p(q), _p(s_g), _p(z_g))
+    _check(rc, "prepack_w4b")
+    return q, s_g.view(np.float16), z_g
+
+
+def linear_w4b(Xq, s_x, X_out, q, s_g, z_g, W_out, m0: int = 0, m1: int | None = None):
+    """Layer output (fp64) with reading-B weights for rows [m0,m1).
+
+    Returns (part int32 [m1-m0, N, K/128] per-group partial sums, y f64 [m1-m0, N])."""
+    lib = _load()
+    Xq = np.ascontiguousarray(Xq, dtype=np.int8)
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    z_g = np.ascontiguousarray(z_g, dtype=np.uint8)
+    s_x = np.ascontiguousarray(s_x, dtype=np.float32)
+    M, K = Xq.shape
+    N = q.shape[0]
+    kp = 0 if X_out is None else X_out.shape[1]
+    xo = _f16bits(X_out) if kp else None
+    wo = _f16bits(W_out) if kp else None
+    m1 = M if m1 is None else m1
+    part = np.empty((m1 - m0, N, K // GROUP), np.int32)
+    y = np.empty((m1 - m0, N), np.float64)
+    rc = lib.oracle_linear_w4b(_p(Xq), _p(s_x), _p(xo), _p(q), _p(_f16bits(s_g)), _p(z_g),
+                               _p(wo), M, N, K, kp, m0, m1, _p(part), _p(y))
+    _check(rc, "linear_w4b")
+    return part, y
+
+
 def quantize_act(X: np.ndarray, idx, T: float):
     """Per-token INT8 activations, outlier gather, detection bitmap, flags.
 

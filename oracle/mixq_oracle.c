@@ -35,6 +35,10 @@
  *     list (outlier locality); detection outside idx is only reported;
  *   - 4-bit level 2 uses integer scale s2 = max(1, ceil((hi-lo)/15)) and zero
  *     z2 = clamp(rint(-lo/s2), 0, 15), with q clamped so (q-z2)*s2 is int8;
+ *   - 4-bit reading B quantizes the fp16 weights per group directly, with a
+ *     real fp16 scale and an integer zero point over a range widened to hold
+ *     0; its layer sums per-group INT32 partials of Xq * (q - z), each scaled
+ *     by its group scale;
  *   - the final Y is evaluated in fp64 (the kernel's fp32 epilogue is checked
  *     against it within the stated tolerance);
  *   - the operation before the layer that the activation pass may absorb is
@@ -182,6 +186,95 @@ int oracle_prepack_w4(const int8_t *Wq8, int N, int K, uint8_t *q, uint8_t *s2, 
         q[at] = (uint8_t)code;
         w8eff[at] = (int8_t)((code - zero) * scale);
       }
+    }
+  }
+  return ORC_OK;
+}
+
+/*
+ * Weight prepack, 4-bit reading B ([MixLLM] "MixLLM: Ein neuer Ansatz": 4-bit
+ * weights quantized asymmetrically per group, 8-bit activations, a two-step
+ * dequantization that keeps the products on INT8 tensor cores, and a fast
+ * integer-to-float conversion of the results).  Unlike reading A there is no
+ * per-row INT8 level: the fp16 weights go to 4 bits directly, with a real
+ * (fp16) scale and an integer zero point per row and group of G = 128 k.
+ * Reading: the two-step dequantization must end in INT8 operands, so the
+ * zero point is an integer subtracted before the product (step 1: q - z in
+ * [-15, 15]); the real scale multiplies the group's INT32 partial sum after
+ * it (step 2, converted to float).  The group range is widened to contain 0,
+ * so z is always one of the 16 codes.  For every row n and group g:
+ *   lo = min(0, min W), hi = max(0, max W)               (fp32, exact)
+ *   s  = fp16( (hi - lo) / 15 )                          (fp32 ops, then fp16)
+ *   if s == 0:  z = 0, q = 0                             (an all-zero group)
+ *   else:       z = clamp(rint(-lo / s), 0, 15)
+ *               q = clamp(rint(W / s) + z, 0, 15)        (s as stored, fp32)
+ * The effective weight is s * (q - z).  Outputs are logical (unpacked):
+ *   q [N][K] u8, s_g [N][K/128] fp16 bits, z_g [N][K/128] u8.
+ */
+int oracle_prepack_w4b(const uint16_t *W, int N, int K, uint8_t *q, uint16_t *s_g,
+                       uint8_t *z_g) {
+  if (N < 0 || K <= 0 || K % ORC_GROUP != 0) return ORC_EINVAL;
+  const int ng = K / ORC_GROUP;
+  for (int n = 0; n < N; ++n) {
+    for (int g = 0; g < ng; ++g) {
+      const uint16_t *w = W + (size_t)n * K + (size_t)g * ORC_GROUP;
+      float lo = 0.0f, hi = 0.0f;
+      for (int i = 0; i < ORC_GROUP; ++i) {
+        float v = h2f(w[i]);
+        if (!isfinite(v)) return ORC_ENONFINITE;
+        if (v < lo) lo = v;
+        if (v > hi) hi = v;
+      }
+      float range = hi - lo;
+      uint16_t s_bits = f2h_bits((double)(range / 15.0f));
+      float s = h2f(s_bits);
+      int zero = 0;
+      if (s > 0.0f) zero = clamp_i32(rint_even(-lo / s), 0, 15);
+      s_g[(size_t)n * ng + g] = s_bits;
+      z_g[(size_t)n * ng + g] = (uint8_t)zero;
+      for (int i = 0; i < ORC_GROUP; ++i) {
+        int code = s > 0.0f ? clamp_i32(rint_even(h2f(w[i]) / s) + zero, 0, 15) : 0;
+        q[(size_t)n * K + (size_t)g * ORC_GROUP + i] = (uint8_t)code;
+      }
+    }
+  }
+  return ORC_OK;
+}
+
+/*
+ * The layer with reading-B weights for rows [m0, m1) ([MixLLM] two-step
+ * dequantization; [MixQ] Fig. 5 + Fig. 12 for the outlier part):
+ *   P[m,n,g] = sum_{k in g} Xq[m,k] * (q[n,k] - z[n,g])     (exact integer)
+ *   y[m,n]   = s_x[m] * sum_g s[n,g] * P[m,n,g]              (fp64)
+ *            + sum_{j < K_out_pad} X_out[m,j] * W_out[n,j]    (fp64)
+ * The activation codes and scales are those of the per-token activation
+ * pass.  part (nullable) is [(m1-m0)][N][K/128]; y is [(m1-m0)][N].
+ */
+int oracle_linear_w4b(const int8_t *Xq, const float *s_x, const uint16_t *X_out,
+                      const uint8_t *q, const uint16_t *s_g, const uint8_t *z_g,
+                      const uint16_t *W_out, int M, int N, int K, int K_out_pad, int m0, int m1,
+                      int32_t *part, double *y) {
+  if (m0 < 0 || m1 > M || m0 > m1 || N < 0 || K <= 0 || K % ORC_GROUP != 0 || K_out_pad < 0)
+    return ORC_EINVAL;
+  const int ng = K / ORC_GROUP;
+#pragma omp parallel for schedule(dynamic, 1)
+  for (int m = m0; m < m1; ++m) {
+    for (int n = 0; n < N; ++n) {
+      double acc = 0.0;
+      for (int g = 0; g < ng; ++g) {
+        int64_t p = 0;
+        const int z = z_g[(size_t)n * ng + g];
+        for (int i = 0; i < ORC_GROUP; ++i) {
+          size_t k = (size_t)g * ORC_GROUP + i;
+          p += (int64_t)Xq[(size_t)m * K + k] * (int64_t)((int)q[(size_t)n * K + k] - z);
+        }
+        if (part) part[((size_t)(m - m0) * N + n) * ng + g] = (int32_t)p;
+        acc += (double)h2f(s_g[(size_t)n * ng + g]) * (double)p;
+      }
+      double o = 0.0;
+      for (int j = 0; j < K_out_pad; ++j)
+        o += (double)h2f(X_out[(size_t)m * K_out_pad + j]) * (double)h2f(W_out[(size_t)n * K_out_pad + j]);
+      y[(size_t)(m - m0) * N + n] = (double)s_x[m] * acc + o;
     }
   }
   return ORC_OK;

@@ -6,7 +6,9 @@ different way (pure-Python brute force, numpy int64/fp64 products), invariants
 that reduce the layer to a simpler textbook computation (no outliers -> plain
 W8A8; every channel an outlier -> the plain fp16 product), a rigorous
 quantization error bound against the exact fp64 product, and exhaustive checks
-of the 4-bit level-2 rules (range, no-overflow, round-trip bound).
+of the 4-bit level-2 rules (range, no-overflow, round-trip bound), and the
+same kinds of checks for the 4-bit reading-B weights (planted codes, round
+trip, dense-product equivalence).
 """
 import json
 import os
@@ -388,3 +390,155 @@ def test_rmsnorm_rejects_bad_eps():
     X = np.ones((1, 8), np.float16)
     with pytest.raises(oracle.OracleError):
         oracle.rmsnorm(X, np.ones(8, np.float16), -1.0)
+
+
+# ------------------------------------------------- 4-bit weights, reading B
+
+def _w4b_eff(q, s_g, z_g):
+    """Effective weights s * (q - z), fp64, groups expanded along k."""
+    s = np.repeat(s_g.astype(np.float64), 128, axis=1)
+    z = np.repeat(z_g.astype(np.float64), 128, axis=1)
+    return s * (q.astype(np.float64) - z)
+
+
+def test_w4b_golden_cases(golden_dir):
+    g = _load(golden_dir, "w4b_cases.json")
+    W = np.zeros((g["rows"], g["K"]), np.float16)
+    for c in g["cases"]:
+        k0 = 128 * c["group"]
+        W[c["row"], k0:k0 + 128] = np.float16(c.get("fill", 0.0))
+        for k, v in c["entries"].items():
+            W[c["row"], k0 + int(k)] = np.float16(v)
+    q, s_g, z_g = oracle.prepack_w4b(W)
+    eff = _w4b_eff(q, s_g, z_g)
+    for c in g["cases"]:
+        r, gi, k0 = c["row"], c["group"], 128 * c["group"]
+        assert int(s_g.view(np.uint16)[r, gi]) == c["s_bits"], c["why"]
+        assert int(z_g[r, gi]) == c["z"], c["why"]
+        for k, qq, e in c["pairs"]:
+            assert q[r, k0 + k] == qq, (c["name"], k, c["why"])
+            assert eff[r, k0 + k] == e, (c["name"], k, eff[r, k0 + k], e)
+
+
+def test_w4b_planted_codes_are_recovered():
+    """Weights built as s0 * (q - z) with codes 0 and 15 in every group give back
+    exactly s0, z and q (s0 varies per group, so a group index mix-up fails)."""
+    rng = np.random.default_rng(21)
+    N, K = 9, 1024
+    ng = K // 128
+    choices = np.array([2.0 ** -8, 3 * 2.0 ** -9, 2.0 ** -4, 5 * 2.0 ** -12, 1.0, 0.75])
+    s0 = choices[rng.integers(0, len(choices), size=(N, ng))]
+    z0 = rng.integers(0, 16, size=(N, ng))
+    q0 = rng.integers(0, 16, size=(N, ng, 128))
+    q0[:, :, rng.integers(0, 128)] = 0
+    q0[:, :, 127 - rng.integers(0, 64)] = 15
+    Wexact = s0[:, :, None] * (q0 - z0[:, :, None])
+    W = Wexact.reshape(N, K).astype(np.float16)
+    assert (W.astype(np.float64) == Wexact.reshape(N, K)).all()  # exact in fp16
+    q, s_g, z_g = oracle.prepack_w4b(W)
+    np.testing.assert_array_equal(s_g.astype(np.float64), s0)
+    np.testing.assert_array_equal(z_g, z0)
+    np.testing.assert_array_equal(q, q0.reshape(N, K))
+    np.testing.assert_array_equal(_w4b_eff(q, s_g, z_g), W.astype(np.float64))
+
+
+def test_w4b_round_trip_bound():
+    """|s (q - z) - W| <= s/2 plus the fp16 rounding of s (relative 2^-11, times
+    at most 15 steps), and the lowest value of a group with a negative entry
+    always takes code 0."""
+    W = np.concatenate([synth.weights(48, 1024), 3.0 * synth.weights(16, 1024, seed=4) + 0.01])
+    W = W.astype(np.float16)
+    q, s_g, z_g = oracle.prepack_w4b(W)
+    assert q.max() <= 15 and z_g.max() <= 15
+    s = np.repeat(s_g.astype(np.float64), 128, axis=1)
+    assert (s_g.astype(np.float64) >= 2.0 ** -14).all()  # normal fp16 scales only
+    err = np.abs(_w4b_eff(q, s_g, z_g) - W.astype(np.float64))
+    eps16 = 2.0 ** -11
+    assert (err <= s * (0.5 + 15 * eps16 / (1 - eps16)) + 1e-12).all()
+    assert (err / s).max() > 0.45  # the bound is close to tight
+    grp = W.reshape(W.shape[0], -1, 128)
+    qg = q.reshape(q.shape[0], -1, 128)
+    neg = grp.min(axis=2) < 0
+    lowest = np.take_along_axis(qg, grp.argmin(axis=2)[:, :, None], axis=2)[:, :, 0]
+    assert neg.any() and (lowest[neg] == 0).all()
+
+
+def test_w4b_one_sided_groups_keep_their_range():
+    """The range is widened to hold 0, so an all-positive group gets z = 0 and an
+    all-negative one z = 15, and neither loses its extreme value to a clamp."""
+    rng = np.random.default_rng(8)
+    pos = rng.uniform(0.5, 2.0, 128).astype(np.float16)
+    W = np.stack([pos, -pos]).astype(np.float16)
+    q, s_g, z_g = oracle.prepack_w4b(W)
+    assert list(z_g[:, 0]) == [0, 15]
+    assert q[0].max() == 15 and q[1].min() == 0
+    err = np.abs(_w4b_eff(q, s_g, z_g) - W.astype(np.float64))
+    assert (err <= s_g.astype(np.float64).max() * 0.51).all()
+
+
+def _w4b_layer_inputs(M, K, N, k_out, seed=0):
+    idx = synth.outlier_channels(K, k_out)
+    X = synth.activations(M, K, idx, synth.channel_factors(k_out)) if k_out else \
+        synth.activations(M, K)
+    W = synth.weights(N, K, seed=seed + 1)
+    Xq, s_x, X_out, _, _ = oracle.quantize_act(X, idx, synth.THRESHOLD)
+    _, _, W_out = oracle.prepack_w8(W, idx)
+    q, s_g, z_g = oracle.prepack_w4b(W)
+    xo = X_out if X_out.shape[1] else None
+    wo = W_out if W_out.shape[1] else None
+    return X, W, Xq, s_x, xo, wo, q, s_g, z_g
+
+
+def test_w4b_layer_brute_force_tiny():
+    """Per-group partial sums and the output, in plain Python integers/floats."""
+    X, W, Xq, s_x, xo, wo, q, s_g, z_g = _w4b_layer_inputs(3, 256, 4, 64)
+    part, y = oracle.linear_w4b(Xq, s_x, xo, q, s_g, z_g, wo)
+    for m in range(3):
+        for n in range(4):
+            acc = 0.0
+            for g in range(2):
+                p = sum(int(Xq[m, k]) * (int(q[n, k]) - int(z_g[n, g]))
+                        for k in range(128 * g, 128 * g + 128))
+                assert part[m, n, g] == p
+                acc += float(s_g[n, g]) * p
+            o = sum(float(xo[m, j]) * float(wo[n, j]) for j in range(xo.shape[1]))
+            want = float(s_x[m]) * acc + o
+            assert abs(y[m, n] - want) <= 1e-12 * (abs(want) + 1.0)
+
+
+@pytest.mark.parametrize("M,K,N,k_out", [(7, 1024, 40, 0), (12, 2048, 24, 32), (5, 512, 64, 130)])
+def test_w4b_layer_equals_dequantized_product(M, K, N, k_out):
+    """The per-group sum equals the product with the dequantized weights
+    s (q - z) written out densely (distributivity), and the partial sums equal
+    the group slices of an int64 matrix product."""
+    X, W, Xq, s_x, xo, wo, q, s_g, z_g = _w4b_layer_inputs(M, K, N, k_out)
+    part, y = oracle.linear_w4b(Xq, s_x, xo, q, s_g, z_g, wo)
+    wint = q.astype(np.int64) - np.repeat(z_g.astype(np.int64), 128, axis=1)
+    for g in range(K // 128):
+        sl = slice(128 * g, 128 * g + 128)
+        np.testing.assert_array_equal(part[:, :, g], Xq[:, sl].astype(np.int64) @ wint[:, sl].T)
+    ref = s_x.astype(np.float64)[:, None] * (Xq.astype(np.float64) @ _w4b_eff(q, s_g, z_g).T)
+    if xo is not None:
+        ref += xo.astype(np.float64) @ wo.astype(np.float64).T
+    np.testing.assert_allclose(y, ref, rtol=1e-11, atol=1e-11)
+
+
+def test_w4b_layer_tracks_the_exact_product():
+    """Against exact X W^T: within the sum of the activation and weight
+    quantization errors term by term, and not vacuously."""
+    M, K, N, k_out = 9, 1024, 32, 16
+    X, W, Xq, s_x, xo, wo, q, s_g, z_g = _w4b_layer_inputs(M, K, N, k_out)
+    _, y = oracle.linear_w4b(Xq, s_x, xo, q, s_g, z_g, wo)
+    x = X.astype(np.float64)
+    w = W.astype(np.float64)
+    ref = x @ w.T
+    xd = s_x.astype(np.float64)[:, None] * Xq.astype(np.float64)  # dequantized dense part
+    xr = x.copy()
+    if xo is not None:  # the outlier part of a mixed token is exact
+        idx = synth.outlier_channels(K, k_out)
+        mixed = np.abs(x).max(axis=1) > synth.THRESHOLD
+        xr[np.ix_(mixed, idx)] = 0.0
+    weff = _w4b_eff(q, s_g, z_g)
+    bound = np.abs(xr - xd) @ np.abs(w).T + np.abs(xd) @ np.abs(weff - w).T
+    assert (np.abs(y - ref) <= bound * (1 + 1e-9) + 1e-12).all()
+    assert np.abs(y - ref).max() < 0.1 * np.abs(ref).max()
