@@ -145,26 +145,42 @@ def _code_only(text: str) -> str:
     return "\n".join(ln.rstrip() for ln in "".join(out).splitlines() if ln.strip())
 
 
-def kernel_source_hash() -> str:
-    """Hash of the code (comments stripped) of every kernel source file: committed ncu
-    counters apply only to this code."""
+# The sources each measured kernel kind is compiled and configured from (its
+# device code, the inline-PTX and tensor-map helpers, the shared constants, and
+# the planner that picks its launch shape).  Committed ncu counters of a kind
+# stay valid while these files' code is unchanged.
+KERNEL_SOURCES = {
+    "quantize": ("quantize.cu", "ptx.cuh", "internal.h"),
+    "quantize_reset": ("quantize.cu", "ptx.cuh", "internal.h"),
+    "gemm_w8": ("gemm.cu", "ptx.cuh", "tma_host.h", "internal.h"),
+    "gemm_w4": ("gemm_w4ts.cu", "gemm.cu", "ptx.cuh", "tma_host.h", "internal.h"),
+    "prepack": ("prepack.cu", "ptx.cuh", "internal.h"),
+}
+
+
+def kernel_source_hash(kind: str | None = None) -> str:
+    """Hash of the code (comments stripped) of the kernel source files: those of one
+    kernel kind, or every file under csrc/ when kind is None."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "mixed_precision_quantized_mixq_b200", "csrc")
-    for f in sorted(os.listdir(csrc)):
-        if f.endswith((".cu", ".cuh", ".h")):
-            with open(os.path.join(csrc, f), encoding="utf-8") as fh:
-                h.update(f.encode() + b"\0" + _code_only(fh.read()).encode())
+    if kind is None:
+        files = sorted(f for f in os.listdir(csrc) if f.endswith((".cu", ".cuh", ".h")))
+    else:
+        files = sorted(KERNEL_SOURCES[kind])
+    for f in files:
+        with open(os.path.join(csrc, f), encoding="utf-8") as fh:
+            h.update(f.encode() + b"\0" + _code_only(fh.read()).encode())
     return h.hexdigest()[:16]
 
 
 def load_traffic(kernel_kind: str, workload: str):
     """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None if the
-    summary is missing or was taken on different kernel sources."""
+    summary is missing or was taken on different sources of that kernel."""
     p = os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)
-        if d.get("source_hash") != kernel_source_hash():
+        if d["source_hashes"][kernel_kind] != kernel_source_hash(kernel_kind):
             return None
         return d["workloads"][workload][kernel_kind]["bytes_per_launch"]
     except Exception:
