@@ -59,8 +59,11 @@ typedef enum mixq_status {
   MIXQ_ERR_NO_DEVICE = 6         /* no usable sm_100 device is current */
 } mixq_status;
 
-/* Weight formats. */
-enum { MIXQ_W8 = 0, MIXQ_W4G128 = 1 };
+/* Weight formats.  MIXQ_W4G128 is the progressive 4-bit format (integer
+ * group scale s2 over per-row INT8 codes, reading A); MIXQ_W4G128_F16S is
+ * the 4-bit format with a real fp16 scale and an integer zero per group
+ * (MixLLM page, "MixLLM: Ein neuer Ansatz", reading B). */
+enum { MIXQ_W8 = 0, MIXQ_W4G128 = 1, MIXQ_W4G128_F16S = 2 };
 
 /* Thread-local text for the last non-OK status returned on this thread. */
 const char *mixq_last_error(void);
@@ -71,8 +74,9 @@ int mixq_version(void);
 /*
  * Sizes of the prepacked weight buffers for mode, N, K, K_out (host only).
  *   *wq_bytes   MIXQ_W8: N*K (int8 codes, tiled, see mixq_prepack_weights).
- *               MIXQ_W4G128: N*K/2 (two 4-bit codes per byte, tiled).
- *   *grp_bytes  MIXQ_W4G128: 4*N*(K/128) (one fp16 pair (s2, z2) per group,
+ *               MIXQ_W4G128, MIXQ_W4G128_F16S: N*K/2 (two 4-bit codes per
+ *               byte, tiled).
+ *   *grp_bytes  4-bit formats: 4*N*(K/128) (one fp16 pair per group,
  *               group-major [K/128][N]); MIXQ_W8: 0.
  *   *wout_bytes 2*N*K_out_pad (fp16 [N][K_out_pad]).
  * Any output pointer may be NULL.
@@ -97,12 +101,22 @@ mixq_status mixq_prepack_size(int mode, int N, int K, int K_out, size_t *wq_byte
  *          16-byte chunk c (K offsets 32c..32c+31) at chunk position
  *          c^((r/2)%4); inside it byte 4w+i holds q at K offset 32c+8w+i in
  *          its low nibble and q at 32c+8w+4+i in its high nibble.
+ *          MIXQ_W4G128_F16S: its 4-bit codes q in the same layout.
  *          mixq_debug_unpack_w8 / _w4 return the logical codes.
- *   s_w    fp32 [N]               a / 127
- *   grp    MIXQ_W4G128 only (else NULL): fp16 pairs (s2, z2) at [g][n], with
- *          s2 = max(1, ceil((hi-lo)/15)), z2 = clamp(rint(-lo/s2), 0, 15) over
- *          the group's INT8 codes, q = clamp(rint(w8/s2)+z2, qlo, qhi) so the
- *          effective weight (q - z2)*s2 always fits int8.
+ *   s_w    fp32 [N]               a / 127 (MIXQ_W4G128_F16S: unused, may be NULL)
+ *   grp    4-bit formats only (else NULL): one fp16 pair per row and group of
+ *          128 K, at [g][n].
+ *          MIXQ_W4G128: (s2, z2) with s2 = max(1, ceil((hi-lo)/15)),
+ *          z2 = clamp(rint(-lo/s2), 0, 15) over the group's INT8 codes, and
+ *          q = clamp(rint(w8/s2)+z2, qlo, qhi) so the effective weight
+ *          (q - z2)*s2 always fits int8.
+ *          MIXQ_W4G128_F16S (MixLLM page, "MixLLM: Ein neuer Ansatz": 4-bit
+ *          asymmetric group-wise weights, two-step dequantization): (s, z)
+ *          straight from the fp16 weights, with lo = min(0, min W) and
+ *          hi = max(0, max W) over the group, s = fp16(fp32(hi - lo) / 15),
+ *          z = clamp(rint(-lo/s), 0, 15), q = clamp(rint(W/s) + z, 0, 15), all
+ *          in fp32; s == 0 (an all-zero group, or a range below the fp16
+ *          range) gives z = q = 0.  The effective weight is s*(q - z).
  *   W_out  fp16 [N][K_out_pad]    W[:, idx[j]] for j < K_out, zero after; may be
  *                                 NULL when K_out == 0.
  */
@@ -220,14 +234,31 @@ mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
                               int ldy, int32_t *status, void *stream);
 
 /*
+ * Same layer with MIXQ_W4G128_F16S weights (MixLLM page, "MixLLM: Ein neuer
+ * Ansatz": two-step dequantization and a fast integer-to-float conversion):
+ *   P[m,n,g] = sum_{k in g} Xq[m,k] (q[n,k] - z[n,g])  (exact INT32 per group
+ *              of 128 K; q - z is the INT8 operand of tcgen05 kind::i8)
+ *   acc[m,n] = sum_g s[n,g] * float(P[m,n,g])          (fp32, groups in K order)
+ *   Y[m,n]   = fp16(acc * s_x[m] + o[m,n])             (o as mixq_gemm_w8a8o16)
+ *   Wq4/grp/W_out from mixq_prepack_weights(MIXQ_W4G128_F16S); the rest as
+ *   mixq_gemm_w8a8o16.  Built for sm_100a and checked by the host-side tests;
+ *   its device parity tests are pending.
+ */
+mixq_status mixq_gemm_w4a8o16_f16s(int M, int N, int K, int K_out, const int8_t *Xq,
+                                   const float *s_x, const void *X_out, const void *Wq4,
+                                   const void *grp, const void *W_out, const int32_t *flags,
+                                   void *Y, int ldy, int32_t *status, void *stream);
+
+/*
  * The launch plan the gemm calls use for a shape (host only, no GPU needed):
  * output tile width *bn in output channels (always 128: MIXQ_W8 tiles are
  * 128 tokens high, two CTAs per SM, token-sized A slots when M <= 64;
  * MIXQ_W4G128 tiles hold all tokens when M <= 64, 128 tokens up to M = 1024,
- * 256 tokens above), the K-split factor *split (thread-block cluster size
- * along K, 1..8; used at M <= 64, and for W4 tiles too few to fill the SMs)
- * and the number of CTAs *ctas.  num_sms <= 0 means "query the current
- * device".
+ * 256 tokens above; MIXQ_W4G128_F16S tiles hold all tokens when M <= 64 and
+ * 64 tokens above, one CTA per SM), the K-split factor *split (thread-block
+ * cluster size along K, 1..8; used at M <= 64, and for 4-bit tiles too few
+ * to fill the SMs) and the number of CTAs *ctas.  num_sms <= 0 means "query
+ * the current device".
  */
 mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, int *split,
                            int *ctas);
@@ -258,7 +289,8 @@ mixq_status mixq_debug_max_active_clusters(int mode, int bn, int split, int smal
 mixq_status mixq_debug_unpack_w8(int N, int K, const void *Wq, int8_t *out, void *stream);
 
 /* Test-only: logical 4-bit codes back from the packed layout:
- * q uint8 [N][K], s2/z2 uint8 [N][K/128]. */
+ * q uint8 [N][K], s2/z2 uint8 [N][K/128] (the grp pair converted to integers;
+ * for MIXQ_W4G128_F16S weights z2 = z, and the real scale is read from grp). */
 mixq_status mixq_debug_unpack_w4(int N, int K, const void *Wq4, const void *grp, uint8_t *q,
                                  uint8_t *s2, uint8_t *z2, int32_t *status, void *stream);
 

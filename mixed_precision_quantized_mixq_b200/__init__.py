@@ -18,7 +18,7 @@ from dataclasses import dataclass
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "libmixq.so")
 
-MIXQ_W8, MIXQ_W4G128 = 0, 1
+MIXQ_W8, MIXQ_W4G128, MIXQ_W4G128_F16S = 0, 1, 2
 STATUS = {0: "MIXQ_OK", 1: "MIXQ_ERR_INVALID_ARG", 2: "MIXQ_ERR_UNSUPPORTED_SHAPE",
           3: "MIXQ_ERR_MISALIGNED", 4: "MIXQ_ERR_CUDA", 5: "MIXQ_ERR_TIMEOUT",
           6: "MIXQ_ERR_NO_DEVICE"}
@@ -40,6 +40,8 @@ _SIGNATURES = {
                                _VP]),
     "mixq_gemm_w4a8o16": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I,
                                _VP, _VP]),
+    "mixq_gemm_w4a8o16_f16s": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I,
+                                    _VP, _VP]),
     "mixq_gemm_plan": (_I, [_I, _I, _I, _I, _I, _c.POINTER(_I), _c.POINTER(_I), _c.POINTER(_I)]),
     "mixq_debug_gemm_i32": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _I, _I, _I, _VP, _VP]),
     "mixq_debug_max_active_clusters": (_I, [_I, _I, _I, _I, _c.POINTER(_I)]),
@@ -140,6 +142,13 @@ def mixq_gemm_w4a8o16(M, N, K, K_out, Xq, s_x, X_out, Wq4, grp, s_w, W_out, flag
                                    Y.stride(0), _ptr(status), _stream(stream)))
 
 
+def mixq_gemm_w4a8o16_f16s(M, N, K, K_out, Xq, s_x, X_out, Wq4, grp, W_out, flags, Y, status,
+                           stream=None):
+    _check(lib().mixq_gemm_w4a8o16_f16s(M, N, K, K_out, _ptr(Xq), _ptr(s_x), _ptr(X_out),
+                                        _ptr(Wq4), _ptr(grp), _ptr(W_out), _ptr(flags), _ptr(Y),
+                                        Y.stride(0), _ptr(status), _stream(stream)))
+
+
 def mixq_gemm_plan(mode: int, M: int, N: int, K: int, num_sms: int = 0):
     bn, split, ctas = _I(), _I(), _I()
     _check(lib().mixq_gemm_plan(mode, M, N, K, num_sms, ctypes.byref(bn), ctypes.byref(split),
@@ -191,9 +200,9 @@ class PackedWeights:
     N: int
     K: int
     idx: "object"      # int32 [K_out]
-    Wq: "object"       # tiled codes: int8 [N*K] (W8) or uint8 [N*K/2] (W4), see mixq.h
-    s_w: "object"      # fp32 [N]
-    grp: "object"      # fp16 [K/128, N, 2] (W4) or None
+    Wq: "object"       # tiled codes: int8 [N*K] (W8) or uint8 [N*K/2] (4-bit), see mixq.h
+    s_w: "object"      # fp32 [N], or None (MIXQ_W4G128_F16S)
+    grp: "object"      # fp16 [K/128, N, 2] group pairs (4-bit) or None
     W_out: "object"    # fp16 [N, K_out_pad] or None
 
     @property
@@ -280,7 +289,7 @@ def prepack(W, idx, mode: int = MIXQ_W8, status=None, stream=None) -> PackedWeig
     else:
         Wq = torch.empty(N * K // 2, dtype=torch.uint8, device=dev)
         grp = torch.empty((K // GROUP, N, 2), dtype=torch.float16, device=dev)
-    s_w = torch.empty(N, dtype=torch.float32, device=dev)
+    s_w = torch.empty(N, dtype=torch.float32, device=dev) if mode != MIXQ_W4G128_F16S else None
     W_out = torch.empty((N, k_out_pad(ko)), dtype=torch.float16, device=dev) if ko else None
     mixq_prepack_weights(mode, W.contiguous(), idx if ko else None, Wq, s_w, grp, W_out, status,
                          stream)
@@ -341,9 +350,12 @@ def gemm(q: QuantAct, w: PackedWeights, Y=None, status=None, stream=None):
     if w.mode == MIXQ_W8:
         mixq_gemm_w8a8o16(M, w.N, K, w.k_out, q.Xq, q.s_x, q.X_out, w.Wq, w.s_w, w.W_out, q.flags,
                           Y, status, stream)
-    else:
+    elif w.mode == MIXQ_W4G128:
         mixq_gemm_w4a8o16(M, w.N, K, w.k_out, q.Xq, q.s_x, q.X_out, w.Wq, w.grp, w.s_w, w.W_out,
                           q.flags, Y, status, stream)
+    else:
+        mixq_gemm_w4a8o16_f16s(M, w.N, K, w.k_out, q.Xq, q.s_x, q.X_out, w.Wq, w.grp, w.W_out,
+                               q.flags, Y, status, stream)
     return Y
 
 

@@ -10,6 +10,7 @@
 #include <string>
 
 #include "../../include/mixq.h"
+#include "gemm_w4b.h"
 #include "internal.h"
 
 namespace {
@@ -106,9 +107,13 @@ const char *mixq_last_error(void) { return g_last_error.c_str(); }
 
 int mixq_version(void) { return 100; }
 
+static bool valid_mode(int mode) {
+  return mode == MIXQ_W8 || mode == MIXQ_W4G128 || mode == MIXQ_W4G128_F16S;
+}
+
 mixq_status mixq_prepack_size(int mode, int N, int K, int K_out, size_t *wq_bytes,
                               size_t *grp_bytes, size_t *wout_bytes) {
-  if (mode != MIXQ_W8 && mode != MIXQ_W4G128) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
+  if (!valid_mode(mode)) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
   mixq_status s = check_shape(0, N, K, K_out);
   if (s != MIXQ_OK) return s;
   const size_t n = static_cast<size_t>(N), k = static_cast<size_t>(K);
@@ -121,14 +126,15 @@ mixq_status mixq_prepack_size(int mode, int N, int K, int K_out, size_t *wq_byte
 mixq_status mixq_prepack_weights(int mode, const void *W, int N, int K, const int32_t *idx,
                                  int K_out, void *Wq, float *s_w, void *grp, void *W_out,
                                  int32_t *status, void *stream) {
-  if (mode != MIXQ_W8 && mode != MIXQ_W4G128) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
+  if (!valid_mode(mode)) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
   mixq_status s = check_shape(0, N, K, K_out);
   if (s != MIXQ_OK) return s;
-  if (!W || !Wq || !s_w) return fail(MIXQ_ERR_INVALID_ARG, "W, Wq and s_w must be non-null");
-  if (mode == MIXQ_W4G128 && !grp) return fail(MIXQ_ERR_INVALID_ARG, "grp must be non-null for MIXQ_W4G128");
+  if (!W || !Wq) return fail(MIXQ_ERR_INVALID_ARG, "W and Wq must be non-null");
+  if (mode != MIXQ_W4G128_F16S && !s_w) return fail(MIXQ_ERR_INVALID_ARG, "s_w must be non-null");
+  if (mode != MIXQ_W8 && !grp) return fail(MIXQ_ERR_INVALID_ARG, "grp must be non-null for 4-bit weights");
   if (K_out > 0 && (!idx || !W_out))
     return fail(MIXQ_ERR_INVALID_ARG, "idx and W_out must be non-null when K_out > 0");
-  if (!aligned16(W) || !aligned16(Wq) || !aligned16(s_w) || (grp && !aligned16(grp)) ||
+  if (!aligned16(W) || !aligned16(Wq) || (s_w && !aligned16(s_w)) || (grp && !aligned16(grp)) ||
       (W_out && !aligned16(W_out)))
     return fail(MIXQ_ERR_MISALIGNED, "matrix pointers must be 16-byte aligned");
   s = check_device(nullptr);
@@ -239,12 +245,12 @@ static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const i
   if (s != MIXQ_OK) return s;
   if (ldy < N || ldy % 8) return fail(MIXQ_ERR_INVALID_ARG, "ldy = %d must be >= N and a multiple of 8", ldy);
   if (M == 0) return check_device(nullptr);
-  if (!Xq || !s_x || !Wq || !s_w || !Y)
+  if (!Xq || !s_x || !Wq || !Y || (mode != MIXQ_W4G128_F16S && !s_w))
     return fail(MIXQ_ERR_INVALID_ARG, "Xq, s_x, Wq, s_w and Y must be non-null");
-  if (mode == MIXQ_W4G128 && !grp) return fail(MIXQ_ERR_INVALID_ARG, "grp must be non-null");
+  if (mode != MIXQ_W8 && !grp) return fail(MIXQ_ERR_INVALID_ARG, "grp must be non-null");
   if (K_out > 0 && (!X_out || !W_out))
     return fail(MIXQ_ERR_INVALID_ARG, "X_out and W_out must be non-null when K_out > 0");
-  if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(Y) || !aligned16(s_w) ||
+  if (!aligned16(Xq) || !aligned16(Wq) || !aligned16(Y) || (s_w && !aligned16(s_w)) ||
       (grp && !aligned16(grp)) || (X_out && !aligned16(X_out)) || (W_out && !aligned16(W_out)))
     return fail(MIXQ_ERR_MISALIGNED, "matrix pointers must be 16-byte aligned");
   int sms = 0;
@@ -269,8 +275,13 @@ static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const i
   a.epi = mixq::Epi::kMixed;
   a.status = status;
   a.wait_limit_ns = kDefaultWaitNs;
-  const mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms);
   const char *why = nullptr;
+  if (mode == MIXQ_W4G128_F16S) {
+    const mixq::GemmPlan plan = mixq::plan_gemm_w4b(M, N, K, sms);
+    const cudaError_t e = mixq::launch_gemm_w4b(a, plan, static_cast<cudaStream_t>(stream), &why);
+    return from_cuda(e, "gemm launch", why);
+  }
+  const mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms);
   const cudaError_t e = mixq::launch_gemm(a, plan, static_cast<cudaStream_t>(stream), &why);
   return from_cuda(e, "gemm launch", why);
 }
@@ -291,16 +302,25 @@ mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
                      ldy, status, stream);
 }
 
+mixq_status mixq_gemm_w4a8o16_f16s(int M, int N, int K, int K_out, const int8_t *Xq,
+                                   const float *s_x, const void *X_out, const void *Wq4,
+                                   const void *grp, const void *W_out, const int32_t *flags,
+                                   void *Y, int ldy, int32_t *status, void *stream) {
+  return gemm_common(MIXQ_W4G128_F16S, M, N, K, K_out, Xq, s_x, X_out, Wq4, grp, nullptr, W_out,
+                     flags, Y, ldy, status, stream);
+}
+
 mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, int *split,
                            int *ctas) {
-  if (mode != MIXQ_W8 && mode != MIXQ_W4G128) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
+  if (!valid_mode(mode)) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);
   mixq_status s = check_shape(M, N, K, 0);
   if (s != MIXQ_OK) return s;
   if (num_sms <= 0) {
     s = check_device(&num_sms);
     if (s != MIXQ_OK) return s;
   }
-  const mixq::GemmPlan p = mixq::plan_gemm(mode, M, N, K, num_sms);
+  const mixq::GemmPlan p = mode == MIXQ_W4G128_F16S ? mixq::plan_gemm_w4b(M, N, K, num_sms)
+                                                   : mixq::plan_gemm(mode, M, N, K, num_sms);
   if (bn) *bn = p.bn;
   if (split) *split = p.split;
   if (ctas) *ctas = p.ctas;

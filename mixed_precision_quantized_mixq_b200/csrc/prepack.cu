@@ -11,6 +11,14 @@
 // effective weight (q - z2) * s2 always fits int8; the GEMM mainloop rebuilds
 // it with one integer multiply-add per four codes.
 //
+// 4-bit reading B (MixLLM page, "MixLLM: Ein neuer Ansatz": asymmetric
+// group-wise 4-bit weights dequantized in two steps onto INT8 tensor cores):
+// no INT8 level; each row and group of 128 along K gets a real fp16 scale s and
+// an integer zero z over a range widened to hold 0, q = clamp(rint(w/s) + z,
+// 0, 15), so that q - z is an INT8 operand and s multiplies the group's INT32
+// partial sum.  The codes share the 4-bit layout below; the group pairs hold
+// (s, z) instead of (s2, z2).
+//
 // Both code layouts are reordered for the GEMM (QServe notes, "compute-aware
 // weight reordering": the layout is chosen so the kernel's loads need no
 // address arithmetic): the weights are cut into tiles of 128 output channels
@@ -183,6 +191,78 @@ __global__ void __launch_bounds__(kPThreads) prepack_kernel(
   }
 }
 
+__device__ __forceinline__ float warp_min_f(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fminf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+// Reading-B prepack: one CTA per weight row (grid-stride), one warp per group
+// of 128 K (four consecutive weights per lane), then the common 4-bit packing.
+// Every decision is taken in fp32 with single IEEE operations in a fixed order:
+//   lo = min(0, min w), hi = max(0, max w)
+//   s  = fp16_rn(fp32(hi - lo) / 15)
+//   z  = s > 0 ? clamp(rint(-lo / s), 0, 15) : 0
+//   q  = s > 0 ? clamp(rint(w / s) + z, 0, 15) : 0
+__global__ void __launch_bounds__(kPThreads) prepack_w4b_kernel(
+    const __half *__restrict__ W, int N, int K, const int32_t *__restrict__ idx, int K_out,
+    int K_out_pad, uint8_t *__restrict__ Wq, __half2 *__restrict__ grp,
+    __half *__restrict__ W_out, int32_t *__restrict__ status) {
+  extern __shared__ int8_t psm[];  // the row's 4-bit codes, one per byte
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int groups = K / kGroup;
+  for (int n = blockIdx.x; n < N; n += gridDim.x) {
+    const __half *wr = W + static_cast<size_t>(n) * K;
+    for (int g = warp; g < groups; g += kPWarps) {
+      const uint2 raw = __ldg(reinterpret_cast<const uint2 *>(wr + g * kGroup) + lane);
+      const float2 f01 = __half22float2(*reinterpret_cast<const __half2 *>(&raw.x));
+      const float2 f23 = __half22float2(*reinterpret_cast<const __half2 *>(&raw.y));
+      const float v[4] = {f01.x, f01.y, f23.x, f23.y};
+      float lo = fminf(fminf(v[0], v[1]), fminf(v[2], v[3]));
+      float hi = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+      lo = fminf(warp_min_f(lo), 0.f);
+      hi = fmaxf(warp_max_f(hi), 0.f);
+      float range = __fsub_rn(hi, lo);
+      if (range <= 0.f) range = 0.f;  // +0 whatever the signs of zero min/max chose
+      const __half s16 = __float2half_rn(__fdiv_rn(range, 15.f));
+      const float s = __half2float(s16);
+      const int z = s > 0.f ? max(0, min(15, __float2int_rn(__fdiv_rn(-lo, s)))) : 0;
+      int8_t *c = psm + g * kGroup + lane * 4;
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        c[i] = static_cast<int8_t>(
+            s > 0.f ? max(0, min(15, __float2int_rn(__fdiv_rn(v[i], s)) + z)) : 0);
+      if (lane == 0) grp[static_cast<size_t>(g) * N + n] = __halves2half2(s16, __int2half_rn(z));
+    }
+    if (K_out_pad > 0) {
+      for (int j = tid; j < K_out_pad; j += kPThreads) {
+        __half v = __ushort_as_half(0);
+        if (j < K_out) {
+          const int c = idx[j];
+          const bool ok = c >= 0 && c < K && (j == 0 || idx[j - 1] < c);
+          if (ok) v = wr[c];
+          else record_error(status, kErrInvalidArg);
+        }
+        W_out[static_cast<size_t>(n) * K_out_pad + j] = v;
+      }
+    }
+    __syncthreads();
+    for (int wi = tid; wi < K / 8; wi += kPThreads) {
+      const int8_t *src = psm + wi * 8;
+      uint32_t word = 0;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint32_t byte = (static_cast<uint32_t>(src[i]) & 0xFu) |
+                              ((static_cast<uint32_t>(src[i + 4]) & 0xFu) << 4);
+        word |= byte << (8 * i);
+      }
+      const int kb = wi >> 4, c = (wi >> 2) & 3, w = wi & 3;
+      *reinterpret_cast<uint32_t *>(Wq + w4_chunk_offset(n, kb, c, K / 128) + 4 * w) = word;
+    }
+    __syncthreads();
+  }
+}
+
 __global__ void unpack_w4_kernel(int N, int K, const uint8_t *__restrict__ Wq4,
                                  const __half2 *__restrict__ grp, uint8_t *__restrict__ q,
                                  uint8_t *__restrict__ s2, uint8_t *__restrict__ z2) {
@@ -246,6 +326,16 @@ cudaError_t launch_prepack(int mode, const void *W, int N, int K, const int32_t 
     prepack_kernel<false><<<grid, kPThreads, 0, stream>>>(
         static_cast<const __half *>(W), N, K, idx, K_out, k_out_pad(K_out), Wq, s_w, nullptr,
         static_cast<__half *>(W_out), status);
+  } else if (mode == 2) {
+    const size_t smem = static_cast<size_t>(K);
+    cudaError_t e = cudaFuncSetAttribute(prepack_w4b_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(smem < 48 * 1024 ? 48 * 1024 : smem));
+    if (e != cudaSuccess) return e;
+    prepack_w4b_kernel<<<grid, kPThreads, smem, stream>>>(
+        static_cast<const __half *>(W), N, K, idx, K_out, k_out_pad(K_out),
+        static_cast<uint8_t *>(Wq), static_cast<__half2 *>(grp), static_cast<__half *>(W_out),
+        status);
   } else {
     const size_t smem = static_cast<size_t>(K);
     cudaError_t e = cudaFuncSetAttribute(prepack_kernel<true>,

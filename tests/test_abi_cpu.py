@@ -176,3 +176,74 @@ def test_gemm_plan_w4(lib, M, N, K):
     else:
         # one CTA per SM, 256-token tiles, no K split
         assert bn == 128 and split == 1 and ctas == -(-M // 256) * (N // 128)
+
+
+# ------------------------------------ 4-bit weights with an fp16 group scale
+
+def test_prepack_size_f16s(lib):
+    # same packed code and group-pair sizes as the progressive 4-bit format
+    for N, K, ko in ((256, 512, 65), (4096, 11008, 64), (128, 128, 0)):
+        assert mq.mixq_prepack_size(mq.MIXQ_W4G128_F16S, N, K, ko) == \
+            mq.mixq_prepack_size(mq.MIXQ_W4G128, N, K, ko)
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 11008, 4096), (16, 4096, 11008),
+                                   (40, 4096, 4096), (64, 256, 1024), (100, 4096, 4096),
+                                   (2048, 11008, 4096), (512, 8192, 28672)])
+def test_gemm_plan_f16s(lib, M, N, K):
+    """One CTA per SM with all tokens (M <= 64) or 64 tokens per tile; a K split
+    only while the tiles leave SMs idle, never past one wave, at most 8 and at
+    most K/128; the smallest split reaching 0.8 CTA per SM with <= 11 K blocks
+    per CTA."""
+    sms, KB = 148, K // 128
+    bn, split, ctas = mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, M, N, K, sms)
+    tiles = -(-M // 64) * (N // 128)
+    assert bn == 128 and ctas == tiles * split
+    assert 1 <= split <= min(8, KB)
+    if split > 1:
+        assert ctas <= sms
+        # no smaller split already met the occupancy and depth goal
+        for s in range(1, split):
+            assert not (tiles * s * 5 >= sms * 4 and -(-KB // s) <= 11)
+        # and the chosen one meets it, or the next one would overflow the wave
+        assert (ctas * 5 >= sms * 4 and -(-KB // split) <= 11) or split == min(8, KB) or \
+            tiles * (split + 1) > sms
+    else:
+        assert tiles * 5 >= sms * 4 or tiles * 2 > sms or KB == 1
+
+
+def test_gemm_plan_f16s_examples(lib):
+    # decode N = 11008: 86 tiles, a second wave would be needed for split 2
+    assert mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, 16, 11008, 4096, 148) == (128, 1, 86)
+    # decode N = 4096, K = 4096: 32 tiles x 4 = 128 CTAs, 8 K blocks each
+    assert mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, 16, 4096, 4096, 148) == (128, 4, 128)
+    # small layer: 4 tiles, split 8 (K = 1024: one K block per CTA)
+    assert mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, 100, 256, 1024, 148) == (128, 8, 32)
+
+
+def test_f16s_host_checks(lib):
+    # the scale-free format takes no s_w: a null s_w passes the host checks (the
+    # call then stops at the missing device), a null Xq or a bad ldy does not
+    g = lib.mixq_gemm_w4a8o16_f16s
+    assert g(4, 256, 256, 0, None, 0x2000, None, 0x3000, 0x4000, None, None, 0x5000, 256, None,
+             None) == 1
+    assert g(4, 256, 256, 0, 0x1000, 0x2000, None, 0x3000, None, None, None, 0x5000, 256, None,
+             None) == 1  # grp missing
+    assert g(4, 256, 256, 0, 0x1000, 0x2000, None, 0x3000, 0x4000, None, None, 0x5000, 250, None,
+             None) == 1
+    assert g(4, 256, 256, 0, 0x1000, 0x2000, None, 0x3008, 0x4000, None, None, 0x5000, 256, None,
+             None) == 3
+    assert g(4, 256, 200, 0, 0x1000, 0x2000, None, 0x3000, 0x4000, None, None, 0x5000, 256, None,
+             None) == 2
+    # prepack: s_w may be null for this format only
+    p = lib.mixq_prepack_weights
+    assert p(mq.MIXQ_W4G128, 0x1000, 256, 256, None, 0, 0x2000, None, 0x3000, None, None,
+             None) == 1
+    assert p(mq.MIXQ_W4G128_F16S, 0x1000, 256, 256, None, 0, 0x2000, None, None, None, None,
+             None) == 1  # grp missing
+    import torch
+    if not torch.cuda.is_available():
+        assert g(4, 256, 256, 0, 0x1000, 0x2000, None, 0x3000, 0x4000, None, None, 0x5000, 256,
+                 None, None) == 6
+        assert p(mq.MIXQ_W4G128_F16S, 0x1000, 256, 256, None, 0, 0x2000, None, 0x3000, None,
+                 None, None) == 6
