@@ -50,7 +50,7 @@ def _worker(rank, world, port, out):
 
 def test_two_gloo_ranks():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a threaded parent
     out = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     t0, g0, idx0, _ = out[0]
@@ -92,7 +92,7 @@ def test_two_gloo_ranks_column_split():
     import synth
     from helpers import oracle_layer
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a threaded parent
     out = mgr.dict()
     mp.spawn(_tp_worker, args=(world, _free_port(), out), nprocs=world, join=True)
     M, K, N, k_out = 8, 512, 512, 16
