@@ -20,7 +20,12 @@ import numpy as np
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "mixq_oracle.c")
 _LIB = os.path.join(_HERE, "libmixq_oracle.so")
+# A planted-mistake build of the oracle (oracle/mutation_check.py) is loaded in
+# place of the real one when this names its shared library.
+_LIB_OVERRIDE = os.environ.get("MIXQ_ORACLE_LIB")
 GROUP = 128
+CFLAGS = ["-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp", "-fPIC", "-shared",
+          "-Wall", "-Wextra"]
 
 _ERRORS = {1: "invalid argument", 2: "non-finite input", 3: "int32 overflow"}
 
@@ -31,10 +36,10 @@ class OracleError(RuntimeError):
 
 def build(force: bool = False) -> str:
     """Compile the oracle with gcc: -O2, no fp contraction, no fast-math, OpenMP."""
+    if _LIB_OVERRIDE:
+        return _LIB_OVERRIDE
     if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
-        cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math", "-fopenmp",
-               "-fPIC", "-shared", "-Wall", "-Wextra", "-o", _LIB, _SRC, "-lm"]
-        subprocess.run(cmd, check=True)
+        subprocess.run(["gcc", *CFLAGS, "-o", _LIB, _SRC, "-lm"], check=True)
     return _LIB
 
 
@@ -45,7 +50,7 @@ def _load():
     global _lib
     if _lib is None:
         build()
-        _lib = ctypes.CDLL(_LIB)
+        _lib = ctypes.CDLL(_LIB_OVERRIDE or _LIB)
     return _lib
 
 
