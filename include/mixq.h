@@ -250,6 +250,13 @@ mixq_status mixq_gemm_w4a8o16_f16s(int M, int N, int K, int K_out, const int8_t 
                                    void *Y, int ldy, int32_t *status, void *stream);
 
 /*
+ * Device workspace the gemm calls need for a shape, in bytes (host only): always
+ * 0.  K-split partial sums are reduced through the distributed shared memory of
+ * a thread-block cluster, so no call takes a workspace argument.
+ */
+size_t mixq_gemm_workspace_size(int M, int N, int K);
+
+/*
  * The launch plan the gemm calls use for a shape (host only, no GPU needed):
  * output tile width *bn in output channels (always 128: MIXQ_W8 tiles are
  * 128 tokens high, two CTAs per SM, token-sized A slots when M <= 64;

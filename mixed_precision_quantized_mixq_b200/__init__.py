@@ -42,6 +42,7 @@ _SIGNATURES = {
                                _VP, _VP]),
     "mixq_gemm_w4a8o16_f16s": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _VP, _I,
                                     _VP, _VP]),
+    "mixq_gemm_workspace_size": (_SZ, [_I, _I, _I]),
     "mixq_gemm_plan": (_I, [_I, _I, _I, _I, _I, _c.POINTER(_I), _c.POINTER(_I), _c.POINTER(_I)]),
     "mixq_debug_gemm_i32": (_I, [_I, _I, _I, _I, _VP, _VP, _VP, _VP, _I, _I, _I, _VP, _VP]),
     "mixq_debug_max_active_clusters": (_I, [_I, _I, _I, _I, _c.POINTER(_I)]),

@@ -310,6 +310,13 @@ mixq_status mixq_gemm_w4a8o16_f16s(int M, int N, int K, int K_out, const int8_t 
                      flags, Y, ldy, status, stream);
 }
 
+size_t mixq_gemm_workspace_size(int M, int N, int K) {
+  (void)M;
+  (void)N;
+  (void)K;
+  return 0;
+}
+
 mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, int *split,
                            int *ctas) {
   if (!valid_mode(mode)) return fail(MIXQ_ERR_INVALID_ARG, "mode = %d", mode);

@@ -39,6 +39,11 @@ def test_version(lib):
     assert lib.mixq_version() == 100
 
 
+def test_no_gemm_workspace(lib):
+    for M, N, K in ((1, 128, 128), (16, 11008, 4096), (8192, 28672, 8192)):
+        assert lib.mixq_gemm_workspace_size(M, N, K) == 0
+
+
 def test_prepack_size(lib):
     assert mq.mixq_prepack_size(mq.MIXQ_W8, 256, 512, 4) == (256 * 512, 0, 2 * 256 * 64)
     assert mq.mixq_prepack_size(mq.MIXQ_W4G128, 256, 512, 65) == (256 * 256, 4 * 256 * 4,
