@@ -146,9 +146,10 @@ mixq_status mixq_prepack_weights(int mode, const void *W, int N, int K, const in
  *                  flags[0] on the device to skip the FP16 slice when no
  *                  token is mixed.
  * K must not exceed 32768 (a token's row is held in registers).
- * For M <= 32 G tokens (G = 2 when K <= 8192, else 1) one thread-block
- * cluster covers the matrix and the call is one kernel; for larger M it is a
- * 1-block reset of bitmap/flags followed by the main pass.
+ * For M <= 16 G tokens (G = 2 when K <= 4096, G = 1 when 4096 < K <= 16384)
+ * one thread-block cluster of at most 16 CTAs covers the matrix and the call
+ * is one kernel; otherwise it is a 1-block reset of bitmap/flags followed by
+ * the main pass.
  */
 mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx, int K_out,
                               float threshold, int8_t *Xq, float *s_x, void *X_out,
