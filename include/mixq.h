@@ -225,7 +225,7 @@ mixq_status mixq_gemm_w8a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
  * expanded back to the INT8 weight (q - z2)*s2, four codes per 32-bit
  * register operation, and multiplied on INT8 tensor cores.  The expanded
  * weights go from registers into tensor memory and are the MMA's A operand
- * (tokens are B), so each CTA owns 128 output channels x up to 128 tokens.
+ * (tokens are B), so each CTA owns 128 output channels x up to 256 tokens.
  *   Wq4/grp/s_w/W_out from mixq_prepack_weights(MIXQ_W4G128); the rest as
  *   mixq_gemm_w8a8o16.
  */
