@@ -147,6 +147,29 @@ def linear_w4b(Xq, s_x, X_out, q, s_g, z_g, W_out, m0: int = 0, m1: int | None =
     return part, y
 
 
+def linear_w4b_points(Xq, s_x, X_out, q, s_g, z_g, W_out, ms, ns):
+    """Reading-B layer output (fp64) and per-group partial sums at sampled points."""
+    lib = _load()
+    Xq = np.ascontiguousarray(Xq, dtype=np.int8)
+    q = np.ascontiguousarray(q, dtype=np.uint8)
+    z_g = np.ascontiguousarray(z_g, dtype=np.uint8)
+    s_x = np.ascontiguousarray(s_x, dtype=np.float32)
+    ms = _idx(ms)
+    ns = _idx(ns)
+    M, K = Xq.shape
+    N = q.shape[0]
+    kp = 0 if X_out is None else X_out.shape[1]
+    xo = _f16bits(X_out) if kp else None
+    wo = _f16bits(W_out) if kp else None
+    part = np.empty((len(ms), K // GROUP), np.int32)
+    y = np.empty(len(ms), np.float64)
+    rc = lib.oracle_linear_w4b_points(_p(Xq), _p(s_x), _p(xo), _p(q), _p(_f16bits(s_g)), _p(z_g),
+                                      _p(wo), M, N, K, kp, _p(ms), _p(ns), len(ms), _p(part),
+                                      _p(y))
+    _check(rc, "linear_w4b_points")
+    return part, y
+
+
 def quantize_act(X: np.ndarray, idx, T: float):
     """Per-token INT8 activations, outlier gather, detection bitmap, flags.
 

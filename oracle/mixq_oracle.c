@@ -281,6 +281,41 @@ int oracle_linear_w4b(const int8_t *Xq, const float *s_x, const uint16_t *X_out,
 }
 
 /*
+ * Same as oracle_linear_w4b, but only at P sampled output points (ms[p],
+ * ns[p]); part (nullable) is [P][K/128], y is [P].
+ */
+int oracle_linear_w4b_points(const int8_t *Xq, const float *s_x, const uint16_t *X_out,
+                             const uint8_t *q, const uint16_t *s_g, const uint8_t *z_g,
+                             const uint16_t *W_out, int M, int N, int K, int K_out_pad,
+                             const int32_t *ms, const int32_t *ns, int P, int32_t *part,
+                             double *y) {
+  if (N < 0 || K <= 0 || K % ORC_GROUP != 0 || K_out_pad < 0 || P < 0) return ORC_EINVAL;
+  for (int i = 0; i < P; ++i)
+    if (ms[i] < 0 || ms[i] >= M || ns[i] < 0 || ns[i] >= N) return ORC_EINVAL;
+  const int ng = K / ORC_GROUP;
+#pragma omp parallel for schedule(static)
+  for (int i = 0; i < P; ++i) {
+    const int m = ms[i], n = ns[i];
+    double acc = 0.0;
+    for (int g = 0; g < ng; ++g) {
+      int64_t sum = 0;
+      const int z = z_g[(size_t)n * ng + g];
+      for (int t = 0; t < ORC_GROUP; ++t) {
+        size_t k = (size_t)g * ORC_GROUP + t;
+        sum += (int64_t)Xq[(size_t)m * K + k] * (int64_t)((int)q[(size_t)n * K + k] - z);
+      }
+      if (part) part[(size_t)i * ng + g] = (int32_t)sum;
+      acc += (double)h2f(s_g[(size_t)n * ng + g]) * (double)sum;
+    }
+    double o = 0.0;
+    for (int j = 0; j < K_out_pad; ++j)
+      o += (double)h2f(X_out[(size_t)m * K_out_pad + j]) * (double)h2f(W_out[(size_t)n * K_out_pad + j]);
+    y[i] = (double)s_x[m] * acc + o;
+  }
+  return ORC_OK;
+}
+
+/*
  * RMS normalisation of each token: the operation before the layer, which the
  * activation pass can absorb ([MixQ] MixQ的解决方案: the amax of quantization
  * can be taken inside the preceding operation).  The pages give no formula for

@@ -542,3 +542,13 @@ def test_w4b_layer_tracks_the_exact_product():
     bound = np.abs(xr - xd) @ np.abs(w).T + np.abs(xd) @ np.abs(weff - w).T
     assert (np.abs(y - ref) <= bound * (1 + 1e-9) + 1e-12).all()
     assert np.abs(y - ref).max() < 0.1 * np.abs(ref).max()
+
+
+def test_w4b_points_match_full():
+    X, W, Xq, s_x, xo, wo, q, s_g, z_g = _w4b_layer_inputs(6, 1024, 40, 16)
+    part, y = oracle.linear_w4b(Xq, s_x, xo, q, s_g, z_g, wo)
+    ms = np.array([0, 5, 3, 3], np.int32)
+    ns = np.array([39, 0, 17, 18], np.int32)
+    p2, y2 = oracle.linear_w4b_points(Xq, s_x, xo, q, s_g, z_g, wo, ms, ns)
+    np.testing.assert_array_equal(p2, part[ms, ns])
+    np.testing.assert_array_equal(y2, y[ms, ns])
