@@ -239,11 +239,13 @@ mixq_status mixq_gemm_w4a8o16(int M, int N, int K, int K_out, const int8_t *Xq, 
  * Ansatz": two-step dequantization and a fast integer-to-float conversion):
  *   P[m,n,g] = sum_{k in g} Xq[m,k] (q[n,k] - z[n,g])  (exact INT32 per group
  *              of 128 K; q - z is the INT8 operand of tcgen05 kind::i8)
- *   acc[m,n] = sum_g s[n,g] * float(P[m,n,g])          (fp32, groups in K order)
+ *   acc[m,n] = sum_g s[n,g] * float(P[m,n,g])          (fp32 fused multiply-adds)
  *   Y[m,n]   = fp16(acc * s_x[m] + o[m,n])             (o as mixq_gemm_w8a8o16)
  *   Wq4/grp/W_out from mixq_prepack_weights(MIXQ_W4G128_F16S); the rest as
- *   mixq_gemm_w8a8o16.  Built for sm_100a and checked by the host-side tests;
- *   its device parity tests are pending.
+ *   mixq_gemm_w8a8o16.  Order of the fp32 sum: without a K split (see
+ *   mixq_gemm_plan) the groups in K order; with a K split over S CTAs each CTA
+ *   sums the groups of its K range in K order and the S partial sums are then
+ *   added in rank order (rank 0 first).
  */
 mixq_status mixq_gemm_w4a8o16_f16s(int M, int N, int K, int K_out, const int8_t *Xq,
                                    const float *s_x, const void *X_out, const void *Wq4,

@@ -4,6 +4,8 @@
 //   P[n,m,g] = sum_{k in g} (q[n,k] - z[n,g]) Xq[m,k]   tcgen05.mma kind::i8,
 //                                                         exact INT32 per group
 //   acc[n,m] = sum_g s[n,g] * float(P[n,m,g])           fp32, groups in K order
+//                                                         (K split: per CTA, then
+//                                                         the CTAs in rank order)
 //   o[n,m]   = sum_j W_out[n,j] X_out[m,j]              tcgen05.mma kind::f16
 //   Y[m,n]   = fp16(acc * s_x[m] + o)
 //

@@ -14,8 +14,7 @@ import oracle
 import synth
 from helpers import Gpu, assert_y_close
 
-pytestmark = [pytest.mark.gpu,
-              pytest.mark.skip(reason="kernels built and host-checked; first device run pending")]
+pytestmark = pytest.mark.gpu
 
 
 @pytest.fixture(scope="module")
