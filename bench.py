@@ -173,10 +173,10 @@ def kernel_source_hash(kind: str | None = None) -> str:
     return h.hexdigest()[:16]
 
 
-def load_traffic(kernel_kind: str, workload: str):
+def load_traffic(kernel_kind: str, workload: str, path: str | None = None):
     """Per-launch DRAM bytes of a kernel from the committed ncu summary, or None if the
     summary is missing or was taken on different sources of that kernel."""
-    p = os.path.join(ROOT, "profiles", "dram_traffic.json")
+    p = path or os.path.join(ROOT, "profiles", "dram_traffic.json")
     try:
         with open(p) as f:
             d = json.load(f)

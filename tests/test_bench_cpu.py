@@ -39,15 +39,33 @@ def test_code_only_strips_comments_not_strings():
     assert '"x // y /* z */"' in out and out.splitlines()[-1] == "  int b;"
 
 
-def test_traffic_is_tied_to_each_kernel_kinds_sources(monkeypatch):
-    # the committed figures were taken on the current sources of the measured kinds
-    for w in ("llama7b-decode", "llama7b-prefill"):
-        for k in ("gemm_w8", "gemm_w4", "quantize"):
-            assert bench.load_traffic(k, w) > 0, (k, w)
-    assert bench.load_traffic("gemm_unknown", "llama7b-decode") is None
+def test_traffic_is_tied_to_each_kernel_kinds_sources(tmp_path, monkeypatch):
+    kinds = ("gemm_w8", "gemm_w4", "quantize")
+    rec = {"source_hashes": {k: bench.kernel_source_hash(k) for k in kinds},
+           "workloads": {"llama7b-decode": {k: {"bytes_per_launch": 1000.0 + i}
+                                            for i, k in enumerate(kinds)}}}
+    p = tmp_path / "traffic.json"
+    p.write_text(json.dumps(rec))
+    # figures taken on the current sources of a kind are returned
+    for i, k in enumerate(kinds):
+        assert bench.load_traffic(k, "llama7b-decode", str(p)) == 1000.0 + i
+    assert bench.load_traffic("gemm_unknown", "llama7b-decode", str(p)) is None
+    assert bench.load_traffic("gemm_w8", "llama7b-prefill", str(p)) is None
     # a change to one kind's sources voids that kind's figure only
     real = bench.kernel_source_hash
     monkeypatch.setattr(bench, "kernel_source_hash",
                         lambda kind=None: "0" * 16 if kind == "gemm_w4" else real(kind))
-    assert bench.load_traffic("gemm_w4", "llama7b-decode") is None
-    assert bench.load_traffic("gemm_w8", "llama7b-decode") > 0
+    assert bench.load_traffic("gemm_w4", "llama7b-decode", str(p)) is None
+    assert bench.load_traffic("gemm_w8", "llama7b-decode", str(p)) == 1000.0
+
+
+def test_committed_traffic_matches_its_recorded_sources():
+    """Each committed figure is reported only while its kind's sources are unchanged."""
+    with open(bench.os.path.join(bench.ROOT, "profiles", "dram_traffic.json")) as f:
+        rec = json.load(f)
+    for w, kinds in rec["workloads"].items():
+        for k, v in kinds.items():
+            if k not in bench.KERNEL_SOURCES:
+                continue
+            fresh = rec["source_hashes"].get(k) == bench.kernel_source_hash(k)
+            assert bench.load_traffic(k, w) == (v["bytes_per_launch"] if fresh else None)
