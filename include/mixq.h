@@ -157,6 +157,37 @@ mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_
                               void *stream);
 
 /*
+ * mixq_quantize_act for callers that cannot allocate device memory.  It has
+ * no counterpart in the pages; it exists for callers that hold only the
+ * layer's own input and output buffers and cannot add a scratch buffer: a
+ * plugin of an inference runtime that is handed fixed, pre-planned buffers,
+ * code whose device memory belongs to another allocator (a framework's
+ * caching allocator or a static arena) that it may not call from here, or a
+ * hot path on which a cudaMalloc, which can synchronize the device, is not
+ * acceptable.  mixq_quantize_act asks the caller for two extra flag words
+ * (flags[2], flags[3]) that its multi-CTA pass uses as a completion ticket;
+ * this entry keeps that ticket in a 256-byte array inside the library
+ * instead, and calls no cudaMalloc, cudaFree or other allocating routine.
+ *   Arguments, outputs and shape limits are those of mixq_quantize_act,
+ *   except flags, which is int32 [2] here ([0] mixed tokens, [1] detected
+ *   channels outside idx; 4-byte aligned).  The scratch needs one word
+ *   whatever the shape, so no shape exceeds it; K > 32768 is rejected with
+ *   MIXQ_ERR_UNSUPPORTED_SHAPE, as by mixq_quantize_act.
+ *   Scratch: int32 [64] (256 bytes) per device, held by every device that
+ *   loads the library until the process exits.  The first call on a device
+ *   looks up the array's device address (cudaGetSymbolAddress, with that
+ *   device current), which can load the library's kernels on it: make that
+ *   first call before any stream capture.  Every call shares the array and
+ *   it keeps the last call's contents; each call clears the ticket before
+ *   using it.  Calls that overlap on the GPU (two streams, or two host
+ *   threads on one device) race on the array: serialise them.
+ */
+mixq_status mixq_quantize_act_static(const void *X, int M, int K, int ldx, const int32_t *idx,
+                                     int K_out, float threshold, int8_t *Xq, float *s_x,
+                                     void *X_out, uint32_t *detect_bitmap, int32_t *flags,
+                                     int32_t *status, void *stream);
+
+/*
  * The activation pass with the preceding RMS normalisation absorbed (MixQ
  * article, MixQ的解决方案: the quantization amax can be taken inside the
  * operation before the layer).  Per token, in fp32 with IEEE division and

@@ -32,6 +32,8 @@ _SIGNATURES = {
     "mixq_prepack_size": (_I, [_I, _I, _I, _I, _c.POINTER(_SZ), _c.POINTER(_SZ), _c.POINTER(_SZ)]),
     "mixq_prepack_weights": (_I, [_I, _VP, _I, _I, _VP, _I, _VP, _VP, _VP, _VP, _VP, _VP]),
     "mixq_quantize_act": (_I, [_VP, _I, _I, _I, _VP, _I, _F, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "mixq_quantize_act_static": (_I, [_VP, _I, _I, _I, _VP, _I, _F, _VP, _VP, _VP, _VP, _VP, _VP,
+                                      _VP]),
     "mixq_rmsnorm_quantize_act": (_I, [_VP, _I, _I, _I, _VP, _F, _VP, _I, _VP, _I, _F, _VP, _VP,
                                        _VP, _VP, _VP, _VP, _VP]),
     "mixq_merge_outliers": (_I, [_VP, _I, _VP, _I, _VP, _c.POINTER(_I)]),
@@ -117,6 +119,17 @@ def mixq_quantize_act(X, idx, threshold, Xq, s_x, X_out, bitmap, flags, status, 
                                    0 if idx is None else idx.numel(), float(threshold), _ptr(Xq),
                                    _ptr(s_x), _ptr(X_out), _ptr(bitmap), _ptr(flags), _ptr(status),
                                    _stream(stream)))
+
+
+def mixq_quantize_act_static(X, idx, threshold, Xq, s_x, X_out, bitmap, flags, status,
+                             stream=None):
+    """mixq_quantize_act with its completion ticket in the library's own static
+    scratch: flags has two words, and the call allocates nothing."""
+    M, K = X.shape
+    _check(lib().mixq_quantize_act_static(_ptr(X), M, K, X.stride(0), _ptr(idx),
+                                          0 if idx is None else idx.numel(), float(threshold),
+                                          _ptr(Xq), _ptr(s_x), _ptr(X_out), _ptr(bitmap),
+                                          _ptr(flags), _ptr(status), _stream(stream)))
 
 
 def mixq_rmsnorm_quantize_act(X, gamma, eps, Xn, idx, threshold, Xq, s_x, X_out, bitmap, flags,

@@ -236,6 +236,35 @@ mixq_status mixq_rmsnorm_quantize_act(const void *X, int M, int K, int ldx, cons
                          flags, status, stream, gamma, eps, Xn, ldxn);
 }
 
+mixq_status mixq_quantize_act_static(const void *X, int M, int K, int ldx, const int32_t *idx,
+                                     int K_out, float threshold, int8_t *Xq, float *s_x,
+                                     void *X_out, uint32_t *detect_bitmap, int32_t *flags,
+                                     int32_t *status, void *stream) {
+  mixq_status s = check_shape(M, 128, K, K_out);
+  if (s != MIXQ_OK) return s;
+  if (K > mixq::quantize_max_k())
+    return fail(MIXQ_ERR_UNSUPPORTED_SHAPE, "K = %d exceeds %d for mixq_quantize_act_static", K,
+                mixq::quantize_max_k());
+  if (ldx < K || ldx % 8) return fail(MIXQ_ERR_INVALID_ARG, "ldx = %d must be >= K and a multiple of 8", ldx);
+  if (!(threshold >= 0.f) || threshold != threshold)
+    return fail(MIXQ_ERR_INVALID_ARG, "threshold must be a finite value >= 0");
+  if (!detect_bitmap || !flags) return fail(MIXQ_ERR_INVALID_ARG, "detect_bitmap and flags must be non-null");
+  if (M > 0 && (!X || !Xq || !s_x)) return fail(MIXQ_ERR_INVALID_ARG, "X, Xq and s_x must be non-null");
+  if (K_out > 0 && !idx) return fail(MIXQ_ERR_INVALID_ARG, "idx must be non-null when K_out > 0");
+  if (K_out > 0 && M > 0 && !X_out) return fail(MIXQ_ERR_INVALID_ARG, "X_out must be non-null when K_out > 0");
+  if ((X && !aligned16(X)) || (Xq && !aligned16(Xq)) || (X_out && !aligned16(X_out)) ||
+      !aligned16(detect_bitmap) || (reinterpret_cast<uintptr_t>(flags) & 3u))
+    return fail(MIXQ_ERR_MISALIGNED,
+                "matrix pointers must be 16-byte aligned and flags 4-byte aligned");
+  int sms = 0;
+  s = check_device(&sms);
+  if (s != MIXQ_OK) return s;
+  return from_cuda(mixq::launch_quantize_act_static(X, M, K, ldx, idx, K_out, threshold, Xq, s_x,
+                                                    X_out, detect_bitmap, flags, status,
+                                                    static_cast<cudaStream_t>(stream), sms),
+                   "quantize (static scratch) launch");
+}
+
 static mixq_status gemm_common(int mode, int M, int N, int K, int K_out, const int8_t *Xq,
                                const float *s_x, const void *X_out, const void *Wq,
                                const void *grp, const float *s_w, const void *W_out,

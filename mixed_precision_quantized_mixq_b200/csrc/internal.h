@@ -26,6 +26,13 @@ cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int3
                                 cudaStream_t stream, int num_sms, const void *gamma = nullptr,
                                 float eps = 0.f, void *Xn = nullptr, int ldxn = 0);
 
+// The same pass with its CTA ticket in the library's static device scratch
+// (flags holds the two output words only); no gamma.
+cudaError_t launch_quantize_act_static(const void *X, int M, int K, int ldx, const int32_t *idx,
+                                       int K_out, float threshold, int8_t *Xq, float *s_x,
+                                       void *X_out, uint32_t *bitmap, int32_t *flags,
+                                       int32_t *status, cudaStream_t stream, int num_sms);
+
 // ----------------------------------------------------------------- prepack
 cudaError_t launch_prepack(int mode, const void *W, int N, int K, const int32_t *idx, int K_out,
                            void *Wq, float *s_w, void *grp, void *W_out, int32_t *status,

@@ -24,8 +24,18 @@
 // grid before their first global memory access.
 #include <cuda_fp16.h>
 
+#include <atomic>
+#include <mutex>
+
 #include "internal.h"
 #include "ptx.cuh"
+
+// Scratch of mixq_quantize_act_static, in the library's own device memory:
+// word 0 is the ticket of the multi-CTA pass (whatever the shape, the pass
+// needs no more); the rest of the 256 bytes is unused.  Every device that
+// loads the library holds one copy until the process exits.
+constexpr int kStaticScratchWords = 64;
+static __device__ __align__(256) int32_t g_quantize_scratch[kStaticScratchWords];
 
 namespace mixq {
 namespace {
@@ -38,6 +48,19 @@ __global__ void reset_detect_kernel(uint32_t *__restrict__ bitmap, int words,
   griddep_wait();
   for (int w = threadIdx.x; w < words; w += blockDim.x) bitmap[w] = 0u;
   if (threadIdx.x < 4) flags[threadIdx.x] = 0;
+  __syncthreads();
+  if (threadIdx.x == 0) griddep_launch_dependents();
+}
+
+// Reset pass of the variant whose CTA ticket lives in the library's static
+// scratch (mixq_quantize_act_static): the two flag words and the ticket.
+__global__ void reset_detect_static_kernel(uint32_t *__restrict__ bitmap, int words,
+                                           int32_t *__restrict__ flags,
+                                           int32_t *__restrict__ ticket) {
+  griddep_wait();
+  for (int w = threadIdx.x; w < words; w += blockDim.x) bitmap[w] = 0u;
+  if (threadIdx.x < 2) flags[threadIdx.x] = 0;
+  if (threadIdx.x == 0) *ticket = 0;
   __syncthreads();
   if (threadIdx.x == 0) griddep_launch_dependents();
 }
@@ -84,6 +107,7 @@ struct QArgs {
   int32_t *flags;
   int32_t *status;
   int cluster_mode;  // one cluster covers the whole grid
+  int32_t *ticket;   // STATIC_TICKET variants: the CTA ticket in the library's scratch
 };
 
 // RT threads per token group (256 for bandwidth-bound shapes; 512 or 1024
@@ -92,7 +116,7 @@ struct QArgs {
 // thread.  NORM: the token is first RMS-normalised in registers
 // (x / sqrt(mean x^2 + eps) * gamma, rounded to fp16 as the normalisation's
 // output would be), so the pass reads X once for both operations.
-template <int VPT, int G, int RT, bool NORM>
+template <int VPT, int G, int RT, bool NORM, bool STATIC_TICKET = false>
 __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   constexpr int kRowWarps = RT / 32;
   extern __shared__ uint32_t qsm[];
@@ -369,8 +393,10 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
       for (int w = 0; w < G * kRowWarps; ++w) t += s_cnt[w];
       a.flags[0] = static_cast<int32_t>(s_mixed_total);
       a.flags[1] = t;
-      a.flags[2] = 0;
-      a.flags[3] = 0;
+      if (!STATIC_TICKET) {
+        a.flags[2] = 0;
+        a.flags[3] = 0;
+      }
     }
     return;
   }
@@ -382,8 +408,9 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   if (tid == 0 && s_part[1]) atomicAdd(reinterpret_cast<int *>(&a.flags[0]), s_part[1]);
   __threadfence();
   __syncthreads();
+  int32_t *const ticket = STATIC_TICKET ? a.ticket : &a.flags[2];
   if (tid == 0) {
-    const int prev = atomicAdd(reinterpret_cast<int *>(&a.flags[2]), 1);
+    const int prev = atomicAdd(reinterpret_cast<int *>(ticket), 1);
     s_last = prev == static_cast<int>(gridDim.x) - 1;
   }
   __syncthreads();
@@ -399,13 +426,17 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
     int total = 0;
     for (int w = 0; w < G * kRowWarps; ++w) total += s_cnt[w];
     a.flags[1] = total;
-    a.flags[2] = 0;
+    *ticket = 0;
   }
 }
 
-template <int VPT, int G, int RT>
+template <int VPT, int G, int RT, bool STATIC_TICKET = false>
 cudaError_t launch_variant(const QArgs &a, int grid, int cluster, cudaStream_t stream) {
-  auto kernel = a.gamma ? quantize_act_kernel<VPT, G, RT, true> : quantize_act_kernel<VPT, G, RT, false>;
+  void (*kernel)(const QArgs);
+  if constexpr (STATIC_TICKET)
+    kernel = quantize_act_kernel<VPT, G, RT, false, true>;
+  else
+    kernel = a.gamma ? quantize_act_kernel<VPT, G, RT, true> : quantize_act_kernel<VPT, G, RT, false>;
   const size_t smem = sizeof(uint32_t) * 3 * (a.K / 32);
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem < 48 * 1024 ? 48 * 1024 : smem));
@@ -429,9 +460,97 @@ cudaError_t launch_variant(const QArgs &a, int grid, int cluster, cudaStream_t s
   return cudaLaunchKernelEx(&cfg, kernel, a);
 }
 
+// Device address of g_quantize_scratch on the current device, looked up once
+// per device (the host-side name is only a stand-in for the device symbol).
+cudaError_t static_scratch(int32_t **out) {
+  static std::atomic<int32_t *> ptr[64];
+  static std::mutex mu;
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  int32_t *p = ptr[dev].load(std::memory_order_acquire);
+  if (!p) {
+    std::lock_guard<std::mutex> lock(mu);
+    p = ptr[dev].load(std::memory_order_acquire);
+    if (!p) {
+      void *q = nullptr;
+      e = cudaGetSymbolAddress(&q, g_quantize_scratch);
+      if (e != cudaSuccess) return e;
+      p = static_cast<int32_t *>(q);
+      ptr[dev].store(p, std::memory_order_release);
+    }
+  }
+  *out = p;
+  return cudaSuccess;
+}
+
 }  // namespace
 
 int quantize_max_k() { return 16 * kRowThreads * 8; }
+
+cudaError_t launch_quantize_act_static(const void *X, int M, int K, int ldx, const int32_t *idx,
+                                       int K_out, float threshold, int8_t *Xq, float *s_x,
+                                       void *X_out, uint32_t *bitmap, int32_t *flags,
+                                       int32_t *status, cudaStream_t stream, int num_sms) {
+  int32_t *ticket = nullptr;
+  cudaError_t e = static_scratch(&ticket);
+  if (e != cudaSuccess) return e;
+  QArgs a{};
+  a.X = static_cast<const __half *>(X);
+  a.M = M;
+  a.K = K;
+  a.ldx = ldx;
+  a.idx = idx;
+  a.K_out = K_out;
+  a.K_out_pad = k_out_pad(K_out);
+  a.T = threshold;
+  a.Xq = Xq;
+  a.s_x = s_x;
+  a.X_out = static_cast<__half *>(X_out);
+  a.bitmap = bitmap;
+  a.flags = flags;
+  a.status = status;
+  a.ticket = ticket;
+  const int nvec = K / 8;
+  // the launch shapes of mixq_quantize_act, with the ticket in the scratch
+  if (M > 0 && M <= 64) {
+    if (nvec <= 512 && (M + 1) / 2 <= kMaxClusterCtas) {
+      a.cluster_mode = 1;
+      return launch_variant<1, 2, 512, true>(a, (M + 1) / 2, (M + 1) / 2, stream);
+    }
+    if (nvec > 512 && nvec <= 2048 && M <= kMaxClusterCtas) {
+      a.cluster_mode = 1;
+      return launch_variant<2, 1, 1024, true>(a, M, M, stream);
+    }
+  }
+  const int vpt_need = (nvec + kRowThreads - 1) / kRowThreads;
+  const int vpt = vpt_need <= 1 ? 1 : vpt_need <= 2 ? 2 : vpt_need <= 4 ? 4 : vpt_need <= 8 ? 8 : 16;
+  {
+    cudaLaunchConfig_t cfg{};
+    cfg.gridDim = dim3(1, 1, 1);
+    cfg.blockDim = dim3(256, 1, 1);
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, reset_detect_static_kernel, bitmap, K / 32, flags, ticket);
+    if (e != cudaSuccess || M == 0) return e;
+  }
+  a.cluster_mode = 0;
+  if (M <= 64 && nvec <= 512) return launch_variant<1, 2, 512, true>(a, (M + 1) / 2, 1, stream);
+  if (M <= 64 && nvec <= 2048) return launch_variant<2, 1, 1024, true>(a, M, 1, stream);
+  const int grid = M < num_sms * 8 ? M : num_sms * 8;
+  switch (vpt) {
+    case 1: return launch_variant<1, 1, kRowThreads, true>(a, grid, 1, stream);
+    case 2: return launch_variant<2, 1, kRowThreads, true>(a, grid, 1, stream);
+    case 4: return launch_variant<4, 1, kRowThreads, true>(a, grid, 1, stream);
+    case 8: return launch_variant<8, 1, kRowThreads, true>(a, grid, 1, stream);
+    default: return launch_variant<16, 1, kRowThreads, true>(a, grid, 1, stream);
+  }
+}
 
 cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx,
                                 int K_out, float threshold, int8_t *Xq, float *s_x, void *X_out,
