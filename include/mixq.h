@@ -345,6 +345,23 @@ mixq_status mixq_debug_gemm_stall(int M, int N, int K, const int8_t *Xq, const v
                                   const float *s_x, const float *s_w, void *Y, int ldy,
                                   uint64_t wait_limit_ns, int32_t *status, void *stream);
 
+/*
+ * Diagnostic: the dense tensor-core rate of this device, measured with the
+ * instruction forms the gemm calls use (no page counterpart; it gives the
+ * tensor-bound GEMMs a peak taken on the same chip in the same run).  One CTA
+ * per SM keeps an A tile (128 x 128 bytes) and a B tile (256 x 128 bytes) in
+ * shared memory, filled with a hashed byte pattern, and one thread issues
+ * `iters` rounds of four back-to-back tcgen05.mma, M = 128, N = 256, into one
+ * tensor-memory accumulator, then waits for them (bounded; a wait that runs
+ * out writes MIXQ_ERR_TIMEOUT to *status).
+ *   kind 0: kind::i8 (s8 x s8 -> s32, K = 32 per MMA)
+ *   kind 1: kind::f16 (f16 x f16 -> f32, K = 16 per MMA)
+ *   iters in [1, 1048576]; *ops (host, non-null) receives the operations one
+ *   launch performs (2 * 128 * 256 * K per MMA, all SMs).  Time the launch
+ *   with events on `stream`; its outputs are discarded.
+ */
+mixq_status mixq_debug_mma_rate(int kind, int iters, double *ops, int32_t *status, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -50,6 +50,7 @@ _SIGNATURES = {
     "mixq_debug_max_active_clusters": (_I, [_I, _I, _I, _I, _c.POINTER(_I)]),
     "mixq_debug_unpack_w8": (_I, [_I, _I, _VP, _VP, _VP]),
     "mixq_debug_unpack_w4": (_I, [_I, _I, _VP, _VP, _VP, _VP, _VP, _VP, _VP]),
+    "mixq_debug_mma_rate": (_I, [_I, _I, _c.POINTER(_c.c_double), _VP, _VP]),
     "mixq_debug_gemm_stall": (_I, [_I, _I, _I, _VP, _VP, _VP, _VP, _VP, _I, _U64, _VP, _VP]),
 }
 
@@ -197,6 +198,15 @@ def mixq_debug_gemm_stall(Xq, Wq, s_x, s_w, Y, wait_limit_ns, status, stream=Non
     _check(lib().mixq_debug_gemm_stall(M, N, K, _ptr(Xq), _ptr(Wq), _ptr(s_x), _ptr(s_w), _ptr(Y),
                                        Y.stride(0), int(wait_limit_ns), _ptr(status),
                                        _stream(stream)))
+
+
+def mixq_debug_mma_rate(kind: int, iters: int, status=None, stream=None) -> float:
+    """Launch the tensor-core rate loop (kind 0 = kind::i8, 1 = kind::f16); returns the
+    operations the launch performs (time it with events on the stream)."""
+    ops = _c.c_double()
+    _check(lib().mixq_debug_mma_rate(kind, iters, ctypes.byref(ops), _ptr(status),
+                                     _stream(stream)))
+    return ops.value
 
 
 # ------------------------------------------------------------ conveniences

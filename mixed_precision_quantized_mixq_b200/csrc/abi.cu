@@ -498,4 +498,18 @@ mixq_status mixq_debug_gemm_stall(int M, int N, int K, const int8_t *Xq, const v
   return from_cuda(e, "stall gemm launch", why);
 }
 
+mixq_status mixq_debug_mma_rate(int kind, int iters, double *ops, int32_t *status, void *stream) {
+  if (kind != 0 && kind != 1) return fail(MIXQ_ERR_INVALID_ARG, "kind = %d must be 0 or 1", kind);
+  if (iters < 1 || iters > (1 << 20))
+    return fail(MIXQ_ERR_INVALID_ARG, "iters = %d must lie in [1, 1048576]", iters);
+  if (!ops) return fail(MIXQ_ERR_INVALID_ARG, "ops must be non-null");
+  int sms = 0;
+  mixq_status s = check_device(&sms);
+  if (s != MIXQ_OK) return s;
+  *ops = mixq::mma_rate_ops_per_launch(kind, iters, sms);
+  return from_cuda(mixq::launch_mma_rate(kind, iters, sms, status, kDefaultWaitNs,
+                                         static_cast<cudaStream_t>(stream)),
+                   "mma rate launch");
+}
+
 }  // extern "C"

@@ -89,6 +89,11 @@ int decode_split(int n_tiles, int KB, int num_sms);
 cudaError_t launch_gemm_w4ts(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
                              const char **why);
 
+// Tensor-core rate loop (mma_rate.cu): kind 0 = kind::i8, 1 = kind::f16.
+double mma_rate_ops_per_launch(int kind, int iters, int num_sms);
+cudaError_t launch_mma_rate(int kind, int iters, int num_sms, int32_t *status,
+                            uint64_t wait_limit_ns, cudaStream_t stream);
+
 // Device properties cached per device.
 int device_sm_count(int dev);
 int device_cc_major(int dev);

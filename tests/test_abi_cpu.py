@@ -252,3 +252,12 @@ def test_f16s_host_checks(lib):
                  None, None) == 6
         assert p(mq.MIXQ_W4G128_F16S, 0x1000, 256, 256, None, 0, 0x2000, None, 0x3000, None,
                  None, None) == 6
+
+
+def test_mma_rate_argument_checks(lib):
+    # host-side checks come before any device access
+    import ctypes as c
+    ops = c.c_double()
+    assert lib.mixq_debug_mma_rate(2, 16, c.byref(ops), None, None) == 1
+    assert lib.mixq_debug_mma_rate(0, 0, c.byref(ops), None, None) == 1
+    assert lib.mixq_debug_mma_rate(0, 16, None, None, None) == 1

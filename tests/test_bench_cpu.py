@@ -69,3 +69,42 @@ def test_committed_traffic_matches_its_recorded_sources():
                 continue
             fresh = rec["source_hashes"].get(k) == bench.kernel_source_hash(k)
             assert bench.load_traffic(k, w) == (v["bytes_per_launch"] if fresh else None)
+
+
+def _bench_cmd(*extra, env=None):
+    import os
+    import subprocess
+    import sys
+    e = dict(os.environ)
+    e.pop("WORLD_SIZE", None)
+    e.pop("RANK", None)
+    e.update(env or {})
+    return subprocess.run([sys.executable, bench.os.path.join(bench.ROOT, "bench.py"), *extra],
+                          capture_output=True, text=True, env=e, timeout=600)
+
+
+def test_gpus_flag_starts_one_process_per_gpu():
+    """--gpus 2 without a launcher runs two ranks (rank 0 prints n_gpus 2), it does not
+    silently run one."""
+    p = _bench_cmd("--impl", "reference", "--gpus", "2", "--workload", "tiny", "--steps", "1",
+                   "--warmup", "3")
+    assert p.returncode == 0, p.stderr[-2000:]
+    lines = [ln for ln in p.stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1
+    assert json.loads(lines[0])["n_gpus"] == 2
+
+
+def test_gpus_flag_must_match_the_launcher():
+    p = _bench_cmd("--impl", "reference", "--gpus", "2", "--workload", "tiny",
+                   env={"WORLD_SIZE": "1", "RANK": "0"})
+    assert p.returncode == 2 and "--gpus 2" in p.stderr
+
+
+def test_workload_modes_and_bytes_of_the_fp16_scale_format():
+    _, cases = bench.workload_cases("llama7b-decode")
+    assert {m for _, ms in cases for m in ms} == {"w8", "w4", "w4b"}
+    _, cases = bench.workload_cases("llama7b-prefill", modes="w4b")
+    assert all(ms == ("w4b",) for _, ms in cases)
+    M, N, K, ko = 16, 4096, 4096, 64
+    # reading-B weights carry no per-row scale s_w
+    assert bench.gemm_bytes("w4", M, N, K, ko) - bench.gemm_bytes("w4b", M, N, K, ko) == 4 * N

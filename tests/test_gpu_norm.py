@@ -70,6 +70,28 @@ def _check(g, Xn, idx, T, what):
     assert list(g["flags"][2:]) == [0, 0], (what, g["flags"])
 
 
+def _check_chain(g, X, gain, idx, T, what):
+    """The whole chain on the oracle side alone, oracle_rmsnorm then oracle_quantize_act,
+    with no value of the kernel as an input: at every token whose scale agrees bit for bit
+    with the chain's, every channel whose normalised value agrees has the same code, and a
+    token whose normalised outlier channels all agree has the same outlier row.  (A token
+    whose amax element lies next to an fp16 rounding boundary may get a scale one step
+    apart; those tokens are covered by the check on the kernel's own normalised values.)"""
+    ref_n = oracle.rmsnorm(X, gain, EPS)
+    Xq, s_x, X_out, _, _ = oracle.quantize_act(ref_n, idx, T)
+    same_s = g["s_x"].view(np.uint32) == s_x.view(np.uint32)
+    same_x = g["Xn"].view(np.uint16) == ref_n.view(np.uint16)
+    mask = same_s[:, None] & same_x
+    if X.shape[0] >= 16:
+        assert same_s.mean() >= 0.8, f"{what}: {same_s.mean():.3f} of the scales agree"
+        assert mask.mean() >= 0.75, f"{what}: {mask.mean():.3f} of the codes compared"
+    np.testing.assert_array_equal(g["Xq"][mask], Xq[mask], err_msg=f"{what}: chain Xq")
+    if len(idx):
+        rows = same_s & same_x[:, np.asarray(idx)].all(axis=1)
+        np.testing.assert_array_equal(g["X_out"][rows].view(np.uint16),
+                                      X_out[rows].view(np.uint16), err_msg=f"{what}: chain X_out")
+
+
 @pytest.mark.parametrize("M,K,k_out", [(1, 4096, 64), (16, 4096, 64), (16, 11008, 64),
                                        (64, 4096, 64), (64, 11008, 64), (130, 4096, 128),
                                        (300, 2048, 32), (16, 256, 4), (7, 28672, 128),
@@ -87,6 +109,8 @@ def test_rmsnorm_quantize_matches_oracle(torch_cuda, M, K, k_out):
     assert (d > 0).mean() < 0.05, f"{(d > 0).mean():.4f} of the values differ by one ulp"
     # every quantization output bit-exact, decided from the kernel's own normalised tokens
     _check(out, out["Xn"], idx, T, f"M{M} K{K} ko{k_out}")
+    # and the oracle's own chain wherever the normalised values agree
+    _check_chain(out, X, g, idx, T, f"M{M} K{K} ko{k_out}")
     # the normalised tokens are an optional output: without them the codes are the same
     out2 = _run(torch_cuda, X, g, idx, T, with_xn=False)
     for k in ("Xq", "s_x", "X_out", "bitmap", "flags"):
