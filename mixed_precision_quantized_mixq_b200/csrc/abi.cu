@@ -383,8 +383,10 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   mixq_status s = check_shape(M, N, K, 0);
   if (s != MIXQ_OK) return s;
   if (ldacc < N || ldacc % 4) return fail(MIXQ_ERR_INVALID_ARG, "ldacc = %d must be >= N and a multiple of 4", ldacc);
-  if (bn != 0 && bn != 32 && bn != 64 && bn != 128 && bn != 256)
+  if (bn != 0 && bn != 32 && bn != 64 && bn != 128 && bn != 256 && bn != 512)
     return fail(MIXQ_ERR_INVALID_ARG, "bn = %d", bn);
+  if (bn == 512 && (mode != MIXQ_W8 || split > 1))
+    return fail(MIXQ_ERR_INVALID_ARG, "bn = 512 (the CTA-pair kernel) takes 8-bit weights and no K split");
   if ((bn == 32 || bn == 64) && M > 64)
     return fail(MIXQ_ERR_INVALID_ARG, "bn = %d needs M <= 64", bn);
   if (split < 0 || split > 8)
@@ -406,7 +408,14 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   if (s != MIXQ_OK) return s;
   mixq::GemmPlan plan = mixq::plan_gemm(mode, M, N, K, sms);
   if (split) plan.split = split;
-  if (mode == MIXQ_W4G128 && (bn == 128 || bn == 256 || (bn == 0 && plan.ts))) {
+  if (bn == 512) {
+    plan.pair = 1;
+  } else if (bn != 0 || split != 0) {
+    plan.pair = 0;
+  }
+  if (plan.pair) {
+    // the CTA-pair kernel
+  } else if (mode == MIXQ_W4G128 && (bn == 128 || bn == 256 || (bn == 0 && plan.ts))) {
     // tensor-memory-operand kernel: bn = 128 the two-CTA-per-SM variant,
     // 256 the one-CTA variant, 0 the planner's choice
     if (bn == 128) plan.small_m = 1;

@@ -364,7 +364,7 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
   const int any_out = outliers_present(p, RAW);
   const bool do_out = any_out && rank == 0;
   if (warp < 4) {
-    if (!mbar_wait(accum_full, 0, p.wait_limit_ns)) fail(s_err, p.status);
+    if (!mbar_wait_sleep(accum_full, 0, p.wait_limit_ns)) fail(s_err, p.status);
     tc_fence_after();
   }
   __syncthreads();
@@ -785,16 +785,25 @@ GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms) {
     const int split = decode_split(n128, K / kBlockK, num_sms);
     return GemmPlan{128, split, n128 * split, 1};
   }
-  // Prefill-sized M: two 128 x 128 CTAs per SM (about 100 KB each), so one
-  // CTA's epilogue overlaps the other's mainloop and the grid packs into waves
-  // twice as finely (measured better than one 128 x 256 CTA per SM, with or
-  // without a K split, on every workload shape).
+  // M >= 256: the persistent CTA-pair kernel (256 x 256 tiles, two SMs per
+  // tile; measured 1.3-1.5x the 128 x 128 kernel on the Llama prefill and 70B
+  // shapes, M = 512..8192, even where its tiles leave pairs idle).
+  const int pairs = num_sms / 2;
+  const int tiles256 = (M + 255) / 256 * ((N + 255) / 256);
+  if (M >= 256) {
+    GemmPlan g{256, 1, 2 * (tiles256 < pairs ? tiles256 : pairs), 0, 0, 1};
+    return g;
+  }
+  // 64 < M < 256: two 128 x 128 CTAs per SM (about 100 KB each), so one CTA's
+  // epilogue overlaps the other's mainloop and the grid packs into waves
+  // twice as finely.
   return GemmPlan{128, 1, (M + kTileM - 1) / kTileM * n128, 1};
 }
 
 cudaError_t launch_gemm(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
                         const char **why) {
   if (a.mode == 1 && plan.ts) return launch_gemm_w4ts(a, plan, stream, why);
+  if (a.mode == 0 && plan.pair) return launch_gemm_pair(a, stream, why);
   const bool w4 = a.mode == 1;
   const bool raw = a.epi == Epi::kRawI32;
 #define MIXQ_DISPATCH(BN_, SM_)                                                      \

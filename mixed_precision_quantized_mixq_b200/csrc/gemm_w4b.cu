@@ -449,7 +449,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   griddep_wait();
   const int any_out = b_outliers_present(p);
   const bool do_out = any_out && rank == 0;
-  if (!mbar_wait(accum_full, 0, p.wait_limit_ns)) b_fail(s_err, p.status);
+  if (!mbar_wait_sleep(accum_full, 0, p.wait_limit_ns)) b_fail(s_err, p.status);
   tc_fence_after();
   __syncthreads();
   const bool failed = *s_err != 0;

@@ -50,6 +50,7 @@ struct GemmPlan {
   int ctas;     // total CTAs launched
   int small_m;  // two-CTA-per-SM kernel variant (half the shared memory and TMEM)
   int ts;       // W4 through the tensor-memory-operand kernel (gemm_w4ts.cu)
+  int pair;     // W8 through the persistent CTA-pair kernel (gemm_pair.cu)
 };
 
 GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms);
@@ -93,6 +94,11 @@ cudaError_t launch_gemm_w4ts(const GemmArgs &a, const GemmPlan &plan, cudaStream
 double mma_rate_ops_per_launch(int kind, int iters, int num_sms);
 cudaError_t launch_mma_rate(int kind, int iters, int num_sms, int32_t *status,
                             uint64_t wait_limit_ns, cudaStream_t stream);
+
+// W8 at large M on CTA pairs (gemm_pair.cu): persistent, 256 x 256 tiles,
+// tcgen05 cta_group::2.  pair_max_active: resident pairs (-1 on error).
+cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t stream, const char **why);
+int pair_max_active(int raw);
 
 // Device properties cached per device.
 int device_sm_count(int dev);

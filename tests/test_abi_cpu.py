@@ -156,6 +156,11 @@ def test_gemm_plan(lib, M, N, K):
     bn, split, ctas = mq.mixq_gemm_plan(mq.MIXQ_W8, M, N, K, 148)
     assert bn in (32, 64, 128, 256) and 1 <= split <= 8 and split <= K // 128
     assert bn >= 128 or M <= 64
+    tiles256 = -(-M // 256) * -(-N // 256)
+    if M >= 256:
+        # persistent CTA-pair kernel: 256 x 256 tiles, one pair per two SMs
+        assert bn == 256 and split == 1 and ctas == 2 * min(tiles256, 74)
+        return
     assert ctas == -(-M // 128) * -(-N // bn) * split
     if M <= 64:
         # decode: narrow tiles and/or a K split across a cluster so that most
