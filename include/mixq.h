@@ -294,10 +294,13 @@ size_t mixq_gemm_workspace_size(int M, int N, int K);
  * The launch plan the gemm calls use for a shape (host only, no GPU needed):
  * output tile width *bn in output channels (MIXQ_W8 at M >= 256: 256, the
  * persistent CTA-pair kernel, 256-token x 256-channel tiles on two SMs each,
- * *ctas = 2 x the pairs it starts; otherwise 128: MIXQ_W8 tiles are 128 tokens
- * high, two CTAs per SM, token-sized A slots when M <= 64;
- * MIXQ_W4G128 tiles hold all tokens when M <= 64, 128 tokens up to M = 1024,
- * 256 tokens above; MIXQ_W4G128_F16S tiles hold all tokens when M <= 64 and
+ * *ctas = 2 x the pairs it starts; MIXQ_W4G128 at M >= 2048: 256, its 4-bit
+ * pair kernel, 256 weight rows x 256 tokens per pair with the weights expanded
+ * into tensor memory; otherwise 128: MIXQ_W8 tiles are 128 tokens high, two
+ * CTAs per SM, token-sized A slots when M <= 64; MIXQ_W4G128 tiles hold all
+ * tokens when M <= 64, 128 tokens up to M = 1024 (256 from M = 256 when
+ * 128-token tiles would leave SMs idle), 256 tokens above; MIXQ_W4G128_F16S
+ * tiles hold all tokens when M <= 64 and
  * 64 tokens above, one CTA per SM), the K-split factor *split (thread-block
  * cluster size along K, 1..8; used at M <= 64, and for 4-bit tiles too few
  * to fill the SMs) and the number of CTAs *ctas.  num_sms <= 0 means "query
@@ -315,8 +318,8 @@ mixq_status mixq_gemm_plan(int mode, int M, int N, int K, int num_sms, int *bn, 
  * variant (a K split only with M <= 64, else MIXQ_ERR_UNSUPPORTED_SHAPE),
  * 256 = its one-CTA-per-SM variant (256-token tiles above M = 1024, where it
  * splits no K), 32/64 = the shared-memory-operand
- * kernel with narrow tiles (M <= 64); 0 = the plan.  bn 512 (MIXQ_W8 only,
- * no K split): the persistent CTA-pair kernel at any M.
+ * kernel with narrow tiles (M <= 64); 0 = the plan.  bn 512 (no K split):
+ * the persistent CTA-pair kernel of the mode at any M.
  */
 mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq, const void *Wq,
                                 const void *grp, int32_t *acc, int ldacc, int bn, int split,

@@ -385,8 +385,8 @@ mixq_status mixq_debug_gemm_i32(int mode, int M, int N, int K, const int8_t *Xq,
   if (ldacc < N || ldacc % 4) return fail(MIXQ_ERR_INVALID_ARG, "ldacc = %d must be >= N and a multiple of 4", ldacc);
   if (bn != 0 && bn != 32 && bn != 64 && bn != 128 && bn != 256 && bn != 512)
     return fail(MIXQ_ERR_INVALID_ARG, "bn = %d", bn);
-  if (bn == 512 && (mode != MIXQ_W8 || split > 1))
-    return fail(MIXQ_ERR_INVALID_ARG, "bn = 512 (the CTA-pair kernel) takes 8-bit weights and no K split");
+  if (bn == 512 && split > 1)
+    return fail(MIXQ_ERR_INVALID_ARG, "bn = 512 (the CTA-pair kernels) takes no K split");
   if ((bn == 32 || bn == 64) && M > 64)
     return fail(MIXQ_ERR_INVALID_ARG, "bn = %d needs M <= 64", bn);
   if (split < 0 || split > 8)

@@ -802,6 +802,7 @@ GemmPlan plan_gemm(int mode, int M, int N, int K, int num_sms) {
 
 cudaError_t launch_gemm(const GemmArgs &a, const GemmPlan &plan, cudaStream_t stream,
                         const char **why) {
+  if (a.mode == 1 && plan.pair) return launch_gemm_pair_w4(a, stream, why);
   if (a.mode == 1 && plan.ts) return launch_gemm_w4ts(a, plan, stream, why);
   if (a.mode == 0 && plan.pair) return launch_gemm_pair(a, stream, why);
   const bool w4 = a.mode == 1;

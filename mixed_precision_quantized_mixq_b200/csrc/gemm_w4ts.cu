@@ -710,14 +710,27 @@ GemmPlan plan_gemm_w4ts(int M, int N, int K, int num_sms) {
     const int split = decode_split(n_tiles, KB, num_sms);
     return GemmPlan{128, split, n_tiles * split, 1, 1};
   }
+  if (M >= 2048) {
+    // the persistent CTA-pair kernel (gemm_pair_w4.cu): 256 weight rows x 256
+    // tokens per pair of SMs (measured 2 % ahead of the one-CTA 256-token
+    // variant at M = 8192, even at 2048; behind it with fewer tiles)
+    const int pairs = num_sms / 2;
+    const int tiles = (M + 255) / 256 * ((N + 255) / 256);
+    GemmPlan g{256, 1, 2 * (tiles < pairs ? tiles : pairs), 0, 0, 1};
+    return g;
+  }
   if (M > 1024) {
     // one CTA per SM with 256-token tiles: half the code bytes per MAC of a
-    // 128-token tile (measured 0-5 % ahead of the two-CTA 128-token variant
-    // and of the smem-operand kernel at M = 2048 and 8192)
+    // 128-token tile
     return GemmPlan{128, 1, (M + 255) / 256 * n_tiles, 0, 1};
   }
   const int m_tiles = (M + 127) / 128;
   const int ctas = m_tiles * n_tiles;
+  if (M >= 256 && ctas * 5 < num_sms * 4) {
+    // too few 128-token tiles to occupy the SMs: 256-token tiles without a K
+    // split (measured 1.5x the split 128-token plan at 512 x 4096 x 4096)
+    return GemmPlan{128, 1, (M + 255) / 256 * n_tiles, 0, 1};
+  }
   if (ctas * 5 < num_sms * 4) {
     // too few 128 x 128 tiles to occupy the SMs: split K over a cluster (the
     // one-CTA variant holds the reduction buffers of 128 tokens)

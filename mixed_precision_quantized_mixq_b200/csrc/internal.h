@@ -99,6 +99,9 @@ cudaError_t launch_mma_rate(int kind, int iters, int num_sms, int32_t *status,
 // tcgen05 cta_group::2.  pair_max_active: resident pairs (-1 on error).
 cudaError_t launch_gemm_pair(const GemmArgs &a, cudaStream_t stream, const char **why);
 int pair_max_active(int raw);
+// W4 (progressive 4-bit) at large M on CTA pairs (gemm_pair_w4.cu): persistent,
+// 256-weight-row x 192-token tiles, weights expanded into tensor memory.
+cudaError_t launch_gemm_pair_w4(const GemmArgs &a, cudaStream_t stream, const char **why);
 
 // Device properties cached per device.
 int device_sm_count(int dev);

@@ -171,8 +171,8 @@ def test_gemm_plan(lib, M, N, K):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 11008, 4096), (64, 4096, 11008),
-                                   (100, 4096, 4096), (512, 4096, 4096), (2048, 11008, 4096),
-                                   (512, 28672, 8192), (512, 8192, 28672)])
+                                   (100, 4096, 4096), (200, 4096, 4096), (512, 4096, 4096),
+                                   (2048, 11008, 4096), (512, 28672, 8192), (512, 8192, 28672)])
 def test_gemm_plan_w4(lib, M, N, K):
     bn, split, ctas = mq.mixq_gemm_plan(mq.MIXQ_W4G128, M, N, K, 148)
     assert 1 <= split <= 8 and split <= K // 128
@@ -180,12 +180,16 @@ def test_gemm_plan_w4(lib, M, N, K):
         # tensor-memory-operand kernel: 128 weight rows x all tokens per tile
         assert bn == 128 and ctas == (N // 128) * split
         assert 64 <= ctas <= 2 * 148
-    elif M <= 1024:
+    elif M >= 2048:
+        # persistent CTA-pair kernel: 256 weight rows x 256 tokens per pair of SMs
+        tiles = -(-M // 256) * -(-N // 256)
+        assert bn == 256 and split == 1 and ctas == 2 * min(tiles, 74)
+    elif M > 1024 or (M >= 256 and -(-M // 128) * (N // 128) * 5 < 148 * 4):
+        # tensor-memory-operand kernel, one CTA per SM with 256-token tiles
+        assert bn == 128 and split == 1 and ctas == -(-M // 256) * (N // 128)
+    else:
         # tensor-memory-operand kernel, 128-token tiles
         assert bn == 128 and ctas == -(-M // 128) * (N // 128) * split
-    else:
-        # one CTA per SM, 256-token tiles, no K split
-        assert bn == 128 and split == 1 and ctas == -(-M // 256) * (N // 128)
 
 
 # ------------------------------------ 4-bit weights with an fp16 group scale
