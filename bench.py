@@ -172,8 +172,9 @@ def _code_only(text: str) -> str:
 KERNEL_SOURCES = {
     "quantize": ("quantize.cu", "ptx.cuh", "internal.h"),
     "quantize_reset": ("quantize.cu", "ptx.cuh", "internal.h"),
-    "gemm_w8": ("gemm.cu", "ptx.cuh", "tma_host.h", "internal.h"),
-    "gemm_w4": ("gemm_w4ts.cu", "gemm.cu", "ptx.cuh", "tma_host.h", "internal.h"),
+    "gemm_w8": ("gemm.cu", "gemm_pair.cu", "ptx.cuh", "tma_host.h", "internal.h"),
+    "gemm_w4": ("gemm_w4ts.cu", "gemm_pair_w4.cu", "gemm.cu", "ptx.cuh", "tma_host.h",
+                "internal.h"),
     "gemm_w4b": ("gemm_w4b.cu", "gemm_w4b.h", "ptx.cuh", "tma_host.h", "internal.h"),
     "prepack": ("prepack.cu", "ptx.cuh", "internal.h"),
 }
@@ -342,10 +343,10 @@ def measure_mma_rate(mq, torch, dev, kind: int, seconds: float, status):
 
 # ----------------------------------------------------------------- GPU arm
 def measure_workload(mq, torch, dev, rank, world, workload, modes, steps, warmup, norm, sampler,
-                     window, before_timed=None, want_e2e=True):
+                     window, before_timed=None, want_e2e=True, case_filter=None):
     """Time one workload: whole-step value, per-kernel-kind durations, end to end.
     Returns a dict of raw measurements (see build_record)."""
-    desc, cases = workload_cases(workload, None, modes)
+    desc, cases = workload_cases(workload, case_filter, modes)
     T = synth.THRESHOLD
     fmt = {"w8": mq.MIXQ_W8, "w4": mq.MIXQ_W4G128, "w4b": mq.MIXQ_W4G128_F16S}
 
@@ -682,7 +683,8 @@ def run_gpu(args, rank, world):
         mq.check_status(st)
 
     main = measure_workload(mq, torch, dev, rank, world, args.workload, args.modes, args.steps,
-                            args.warmup, args.norm, sampler, "main", before_timed=int8_peak)
+                            args.warmup, args.norm, sampler, "main", before_timed=int8_peak,
+                            case_filter=args.case)
     i8 = peak_info["i8"]["median"]
     rule = (f"measured in this run: the library's tcgen05.mma kind::i8 rate loop (M=128, N=256, "
             f"K=32 per MMA, operands resident in shared memory, one CTA per SM), median of "
