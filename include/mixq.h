@@ -31,8 +31,9 @@
  *   - Kernels are launched with programmatic dependent launch: a call's
  *     kernels may begin while the preceding kernel on the stream finishes, and
  *     wait for it before reading its outputs.  The gemm calls start streaming
- *     the prepacked weights (Wq, grp) before that wait, so those buffers must
- *     not be written by the kernel immediately preceding the gemm call.
+ *     the prepacked weights (Wq, grp) before that wait, and the activation
+ *     passes read the outlier list idx before it, so those buffers must not be
+ *     written by the kernel immediately preceding the call.
  *
  * Shape rules (MIXQ_ERR_UNSUPPORTED_SHAPE otherwise): K % 128 == 0, K > 0,
  * N % 128 == 0, N > 0, M >= 0, 0 <= K_out <= K.  K_out_pad is K_out rounded up

@@ -21,7 +21,8 @@
 //     them with atomics, and the last CTA to finish (ticket in flags[2])
 //     counts the detections outside the outlier list.
 // All kernels use programmatic dependent launch: they wait for the preceding
-// grid before their first global memory access.
+// grid before touching X, the outputs or the status word (the main pass reads
+// the outlier list and builds its bitset before that wait).
 #include <cuda_fp16.h>
 
 #include <atomic>
@@ -133,20 +134,10 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   const int nvec = a.K >> 3;  // 8 fp16 per 16-byte vector
   const int row_stride = gridDim.x * G;
 
-  griddep_wait();
-  // Start this group's first token load before the outlier bitset is built
-  // so the two latencies overlap.
-  int m = blockIdx.x * G + g;
-  uint4 v[VPT];
-#pragma unroll
-  for (int i = 0; i < VPT; ++i) {
-    const int vi = gt + i * RT;
-    v[i] = (m < a.M && vi < nvec)
-               ? __ldg(reinterpret_cast<const uint4 *>(a.X + static_cast<size_t>(m) * a.ldx) + vi)
-               : make_uint4(0u, 0u, 0u, 0u);
-  }
-  // The first outlier index of this thread is read alongside the token row
-  // (both latencies overlap); any further ones below.
+  // The outlier list does not come from the preceding kernel: its bitset and
+  // rank prefix are built before waiting for that kernel, so under
+  // programmatic dependent launch this part overlaps the preceding kernel.
+  if (tid == 0) griddep_launch_dependents();
   int c_first = -1, c_prev = -1;
   if (tid < a.K_out) {
     c_first = a.idx[tid];
@@ -190,9 +181,16 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
     }
   }
   __syncthreads();
-  if (tid == 0) {
-    if (s_bad) record_error(a.status, kErrInvalidArg);
-    griddep_launch_dependents();
+  griddep_wait();
+  if (tid == 0 && s_bad) record_error(a.status, kErrInvalidArg);
+  int m = blockIdx.x * G + g;
+  uint4 v[VPT];
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int vi = gt + i * RT;
+    v[i] = (m < a.M && vi < nvec)
+               ? __ldg(reinterpret_cast<const uint4 *>(a.X + static_cast<size_t>(m) * a.ldx) + vi)
+               : make_uint4(0u, 0u, 0u, 0u);
   }
 
   // The group's next token is loaded while this one is processed (when the
