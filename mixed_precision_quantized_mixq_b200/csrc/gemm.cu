@@ -239,9 +239,13 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
       for (int j = 0; j < pre; ++j)
         tma_load_2d(a_slot(j), &tm_a, &full[j], (kb_begin + j) * kBlockK, m0, pol_a);
       int issued = pre;
+      int s = pre == stages ? 0 : pre;
+      uint32_t ph = pre == stages ? 1u : 0u;
       for (int j = pre; j < njobs; ++j) {
-        const int s = j % stages;
-        const uint32_t ph = (j / stages) & 1;
+        if (j > pre && ++s == stages) {
+          s = 0;
+          ph ^= 1u;
+        }
         if (!mbar_wait(&empty[s], ph ^ 1, p.wait_limit_ns)) {
           fail(s_err, p.status);
           break;
@@ -267,20 +271,26 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
       constexpr uint32_t kIdF16 = idesc_f16_f32(kTileM, BN);
       const uint32_t t_i32 = tmem_base;
       const uint32_t t_f32 = tmem_base + BN;
+      // This thread's per-job path bounds a decode-sized CTA (its MMAs are
+      // short): the ring position advances incrementally, and a stage's
+      // descriptors are those of stage 0 plus a fixed start-address offset.
+      const uint64_t ad0 = sw128_kmajor_desc(smem_u32(a_slot(0)));
+      const uint64_t bd0 = sw128_kmajor_desc(smem_u32(b_slot(0)));
+      const uint64_t a_step = static_cast<uint64_t>(p.a_stride >> 4);
+      constexpr uint64_t b_step = static_cast<uint64_t>(C::kBStage >> 4);
+      uint64_t *const gate = W4 ? ready : full;
       griddep_wait();
       const int n_out = (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
       const int njobs = p.debug_stall ? 1 : n_i8 + n_out;
-      int consumed = 0;
-      for (int j = 0; j < njobs; ++j) {
-        const int s = j % stages;
-        const uint32_t ph = (j / stages) & 1;
-        if (!mbar_wait(W4 ? &ready[s] : &full[s], ph, p.wait_limit_ns)) {
+      int s = 0, j = 0;
+      uint32_t ph = 0;
+      uint64_t ad = ad0, bd = bd0;
+      for (; j < njobs; ++j) {
+        if (!mbar_try_wait(&gate[s], ph) && !mbar_wait(&gate[s], ph, p.wait_limit_ns)) {
           fail(s_err, p.status);
           break;
         }
         tc_fence_after();
-        const uint64_t ad = sw128_kmajor_desc(smem_u32(a_slot(s)));
-        const uint64_t bd = sw128_kmajor_desc(smem_u32(b_slot(s)));
         if (j < n_i8) {
 #pragma unroll
           for (int k = 0; k < 4; ++k)
@@ -291,10 +301,18 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
             mma_f16(t_f32, ad + 2 * k, bd + 2 * k, kIdF16, (j > n_i8 || k > 0) ? 1u : 0u);
         }
         mma_commit(&empty[s]);
-        consumed = j + 1;
+        if (++s == stages) {
+          s = 0;
+          ph ^= 1u;
+          ad = ad0;
+          bd = bd0;
+        } else {
+          ad += a_step;
+          bd += b_step;
+        }
       }
       mma_commit(accum_full);
-      s_misc[2] = consumed;
+      s_misc[2] = j;
     }
   } else if ((warp == 2 || warp == 3) && !RAW) {
     // ------------------------------------ token scales of the tile, early
@@ -491,7 +509,8 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
     const int c4n = (c_end - c_begin) / 4;
 #pragma unroll 1
     for (int r = 0; r < BN / C::kCW; ++r) {
-      if (warp < 4 && !failed) {
+      // only the warps whose TMEM lanes hold token rows read the accumulators
+      if (warp < 4 && warp * 32 < rows_valid && !failed) {
         const int row = warp * 32 + lane;
 #pragma unroll 1
         for (int c = 0; c < C::kCW / 32; ++c) {

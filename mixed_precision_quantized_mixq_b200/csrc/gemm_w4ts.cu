@@ -310,6 +310,9 @@ __global__ void __launch_bounds__(kTsThreads, TsCfg<SM>::kMinBlocks)
     if (lane == 0) {
       const uint32_t id_i8 = idesc_s8_s32(128, bt);
       const uint32_t id_f16 = idesc_f16_f32(128, bt);
+      // token-tile descriptor of stage 0; stage s adds a fixed start-address offset
+      const uint64_t bd0 = sw128_kmajor_desc(smem_u32(stage(0) + p.w_slot));
+      const uint64_t st_step = static_cast<uint64_t>(p.stage_bytes >> 4);
       griddep_wait();
       const int n_out = (ts_outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kTsOutK : 0;
       const int njobs = n_i8 + n_out;
@@ -324,7 +327,7 @@ __global__ void __launch_bounds__(kTsThreads, TsCfg<SM>::kMinBlocks)
           }
           tc_fence_after();
           const uint32_t ta = t_a + ra.slot * a_cols;
-          const uint64_t bd = sw128_kmajor_desc(smem_u32(stage(s) + p.w_slot));
+          const uint64_t bd = bd0 + static_cast<uint64_t>(s) * st_step;
           const int nkb = job_nkb(j);
           for (int kk = 0; kk < nkb; ++kk) {
             const uint64_t bdk = bd + static_cast<uint64_t>(kk * tok_bytes >> 4);
