@@ -301,8 +301,8 @@ size_t mixq_gemm_workspace_size(int M, int N, int K);
  * CTAs per SM, token-sized A slots when M <= 64; MIXQ_W4G128 tiles hold all
  * tokens when M <= 64, 128 tokens up to M = 1024 (256 from M = 256 when
  * 128-token tiles would leave SMs idle), 256 tokens above; MIXQ_W4G128_F16S
- * tiles hold all tokens when M <= 64 and
- * 64 tokens above, one CTA per SM), the K-split factor *split (thread-block
+ * tiles hold all tokens when M <= 64 (two CTAs per SM when M <= 16, else one)
+ * and 64 tokens above, one CTA per SM), the K-split factor *split (thread-block
  * cluster size along K, 1..8; used at M <= 64, and for 4-bit tiles too few
  * to fill the SMs) and the number of CTAs *ctas.  num_sms <= 0 means "query
  * the current device".

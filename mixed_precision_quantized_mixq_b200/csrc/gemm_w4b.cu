@@ -26,8 +26,11 @@
 // subtracts that float: the floats in [2^23, 2^24) are exactly the integers,
 // so the result is exact for |P| < 2^22 (here |P| <= 128 * 127 * 15).
 //
-// One CTA per SM (384 threads, 512 TMEM columns) computes a 128-weight-row x
-// BT-token tile (BT = 16..64) over a K range:
+// One CTA (384 threads) computes a 128-weight-row x BT-token tile over a K
+// range: one CTA per SM with 512 TMEM columns and BT = 16..64, or, for at most
+// 16 tokens, two per SM with 256 columns and half the shared memory each (the
+// decode variant: a K split of its few tiles over clusters then keeps about a
+// CTA per SM streaming weights):
 //   warp 0 lane 0   producer: packed codes + (s, z) pairs by bulk copy, token
 //                   tiles by TMA (128-byte swizzle), outlier stages (W_out and
 //                   X_out tiles, 64-byte swizzle)
@@ -63,11 +66,23 @@ constexpr int kBWOut = 128 * kBOutK * 2;        // W_out tile of an outlier stag
 constexpr int kBMaxTokens = 64;                 // tokens per tile (MMA N) at most
 constexpr int kBExtra = 1024 + 4 * kBMaxTokens;  // barriers, s_x[BT]
 constexpr int kBPitch = 128 + 4;                 // floats per token row of a partial tile
-constexpr int kBSmemMax = 232448;                // one CTA per SM
-constexpr int kBTmemCols = 512;
-constexpr int kBPartCol = 64;  // INT32 partial tile b at TMEM column 64 b
-constexpr int kBF32Col = 128;  // FP32 outlier accumulator
-constexpr int kBACol = 256;    // first column of the TMEM A ring
+constexpr int kBSmallMaxTokens = 16;             // tokens per tile of the two-CTA variant
+
+// One CTA per SM (512 TMEM columns, all of shared memory), or -- SM2, decode-
+// sized M -- two per SM with half of each, so that a K split of the few
+// output tiles still has one CTA per SM beside it (and a CTA of the next
+// kernel can start there).  TMEM: INT32 partial tile b at column kPartCol b,
+// the FP32 outlier accumulator at kF32Col, the A ring from kACol.
+template <bool SM2>
+struct BCfg {
+  static constexpr int kMinBlocks = SM2 ? 2 : 1;
+  static constexpr int kSmemMax = SM2 ? 233472 / 2 - 1024 : 232448;
+  static constexpr int kTmemCols = SM2 ? 256 : 512;
+  static constexpr int kPartCol = SM2 ? 32 : 64;
+  static constexpr int kF32Col = SM2 ? 64 : 128;
+  static constexpr int kACol = SM2 ? 128 : 256;
+  static constexpr int kMaxTokens = SM2 ? kBSmallMaxTokens : kBMaxTokens;
+};
 
 // Stage layout as in reading A's kernel: [codes: kbpj x 8 KB][pairs: kbpj x
 // 512 B] padded to 1 KB (= w_slot), then the token tiles [kbpj][BT x 128 B].
@@ -150,19 +165,21 @@ struct BRing {
   }
 };
 
-template <int NCH>
-__global__ void __launch_bounds__(kBThreads, 1)
+template <int NCH, bool SM2>
+__global__ void __launch_bounds__(kBThreads, BCfg<SM2>::kMinBlocks)
     mixq_w4b_kernel(const __grid_constant__ CUtensorMap tm_a,   // Xq [M][K] int8, box {128, BT}
                     const __grid_constant__ CUtensorMap tm_xo,  // X_out [M][K_out_pad], box {32, BT}
                     const __grid_constant__ CUtensorMap tm_wo,  // W_out [N][K_out_pad], box {32, 128}
                     const __grid_constant__ CUtensorMap tm_y,   // Y [M][ldy] fp16, box {64, BT}
                     const BParams p) {
+  using C = BCfg<SM2>;
   constexpr int BT = 16 * NCH;
+  static_assert(BT <= C::kMaxTokens && BT <= C::kPartCol, "token tile of the variant");
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const int stages = p.stages;
-  const int kbpj = p.kbpj;
+  const int kbpj = SM2 ? 1 : p.kbpj;  // SM2: one K block per job (register budget)
   auto stage = [&](int s) { return smem + s * p.stage_bytes; };
   uint8_t *extra = smem + stages * p.stage_bytes;
   uint64_t *bars = reinterpret_cast<uint64_t *>(extra);
@@ -234,7 +251,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
     }
   }
   if (warp == 1) {
-    tmem_alloc(tmem_holder, kBTmemCols);
+    tmem_alloc(tmem_holder, C::kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -243,8 +260,8 @@ __global__ void __launch_bounds__(kBThreads, 1)
   if (threadIdx.x == 0) griddep_launch_dependents();
   const uint32_t tmem_base = *tmem_holder;
   const uint32_t t_part = tmem_base;
-  const uint32_t t_f32 = tmem_base + kBF32Col;
-  const uint32_t t_a = tmem_base + kBACol;
+  const uint32_t t_f32 = tmem_base + C::kF32Col;
+  const uint32_t t_a = tmem_base + C::kACol;
   const uint32_t a_cols = 32u * kbpj;
   int *s_err = &s_misc[0];
   float acc[BT];  // drain warps: fp32 sums of the thread's weight row
@@ -322,7 +339,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
             const uint64_t bdk = bd + static_cast<uint64_t>(kk * tok_bytes >> 4);
 #pragma unroll
             for (int k = 0; k < 4; ++k)
-              mma_i8_ts(t_part + b * kBPartCol, ta + kk * 32 + k * 8, bdk + 2 * k, id_i8,
+              mma_i8_ts(t_part + b * C::kPartCol, ta + kk * 32 + k * 8, bdk + 2 * k, id_i8,
                         k > 0 ? 1u : 0u);
             mma_commit(&part_full[b]);
           }
@@ -430,7 +447,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
       tc_fence_after();
       uint32_t v[NCH][16];
 #pragma unroll
-      for (int c = 0; c < NCH; ++c) tmem_ld16(t_part + b * kBPartCol + lane_addr + c * 16, v[c]);
+      for (int c = 0; c < NCH; ++c) tmem_ld16(t_part + b * C::kPartCol + lane_addr + c * 16, v[c]);
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
@@ -573,7 +590,7 @@ __global__ void __launch_bounds__(kBThreads, 1)
   }
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem_base, kBTmemCols);
+    tmem_dealloc(tmem_base, C::kTmemCols);
   }
 }
 
@@ -587,34 +604,38 @@ int b_tokens(int M) {
   return bt < 16 ? 16 : bt;
 }
 
+template <bool SM2>
 BGeometry b_geometry(int M) {
+  using C = BCfg<SM2>;
   BGeometry g{};
   g.bt = b_tokens(M);
-  // two K blocks per job unless that leaves fewer than three stages
-  for (int kbpj = 2; kbpj >= 1; --kbpj) {
+  // two K blocks per job unless that leaves fewer than three stages; the
+  // two-CTA variant takes one (its expansion threads have 80 registers)
+  for (int kbpj = SM2 ? 1 : 2; kbpj >= 1; --kbpj) {
     g.kbpj = kbpj;
     g.w_slot = (kbpj * (kBPacked + kBGrp) + 1023) / 1024 * 1024;
     g.stage_bytes = g.w_slot + kbpj * g.bt * kBlockK;
-    g.stages = (kBSmemMax - 1024 - kBExtra) / g.stage_bytes;
+    g.stages = (C::kSmemMax - 1024 - kBExtra) / g.stage_bytes;
     if (g.stages > kBMaxStages) g.stages = kBMaxStages;
     if (g.stages >= 3) break;
   }
-  g.a_stages = (kBTmemCols - kBACol) / (32 * g.kbpj);
+  g.a_stages = (C::kTmemCols - C::kACol) / (32 * g.kbpj);
   if (g.a_stages > g.stages) g.a_stages = g.stages;
   g.smem = g.stages * g.stage_bytes + kBExtra + 1024;
   return g;
 }
 
-template <int NCH>
+template <int NCH, bool SM2>
 cudaError_t launch_b_variant(const GemmArgs &a, const GemmPlan &plan, const BGeometry &geo,
                              cudaStream_t stream, const char **why) {
+  using C = BCfg<SM2>;
   static std::atomic<uint64_t> smem_done{0};
-  auto kernel = mixq_w4b_kernel<NCH>;
-  cudaError_t e = ensure_smem(kernel, kBSmemMax, smem_done);
+  auto kernel = mixq_w4b_kernel<NCH, SM2>;
+  cudaError_t e = ensure_smem(kernel, C::kSmemMax, smem_done);
   if (e != cudaSuccess) return e;
   const int red_bytes = 2 * geo.bt * kBPitch * 4;
   if (geo.bt != 16 * NCH || geo.stages < 2 || geo.stages < geo.a_stages ||
-      geo.a_stages > kBMaxStages || geo.smem > kBSmemMax || geo.w_slot < kBWOut ||
+      geo.a_stages > kBMaxStages || geo.smem > C::kSmemMax || geo.w_slot < kBWOut ||
       plan.split < 1 || plan.split > 8 || plan.split > a.K / kBlockK ||
       (plan.split > 1 && geo.stages * geo.stage_bytes < red_bytes) ||
       (plan.split == 1 && geo.stages * geo.stage_bytes < 2 * geo.bt * 128)) {
@@ -681,12 +702,19 @@ cudaError_t launch_b_variant(const GemmArgs &a, const GemmPlan &plan, const BGeo
 }  // namespace
 
 GemmPlan plan_gemm_w4b(int M, int N, int K, int num_sms) {
-  // One CTA per SM.  While the output tiles leave SMs idle, split K over a
-  // cluster: the smallest split giving at least 0.8 CTA per SM with at most
-  // 11 K blocks per CTA, else the largest that still fits one wave.
   const int KB = K / kBlockK;
   const int bt = b_tokens(M);
   const int tiles = (M + bt - 1) / bt * (N / 128);
+  if (M <= kBSmallMaxTokens) {
+    // decode-sized M: the two-CTA variant, K split as for the other decode
+    // kernels (about 10 K blocks per CTA once ~0.8 CTA per SM stream, at
+    // most two CTAs per SM)
+    const int split = decode_split(tiles, KB, num_sms);
+    return GemmPlan{128, split, tiles * split, 1, 0};
+  }
+  // One CTA per SM.  While the output tiles leave SMs idle, split K over a
+  // cluster: the smallest split giving at least 0.8 CTA per SM with at most
+  // 11 K blocks per CTA, else the largest that still fits one wave.
   int best = 1;
   for (int s = 1; s <= 8 && s <= KB; ++s) {
     if (s > 1 && tiles * s > num_sms) break;
@@ -702,16 +730,23 @@ cudaError_t launch_gemm_w4b(const GemmArgs &a, const GemmPlan &plan, cudaStream_
     *why = "the reading-B GEMM has no raw accumulator output";
     return cudaErrorInvalidValue;
   }
-  const BGeometry geo = b_geometry(a.M);
+  if (plan.small_m) {
+    if (a.M > kBSmallMaxTokens) {
+      *why = "the two-CTA reading-B variant takes at most 16 tokens";
+      return cudaErrorInvalidValue;
+    }
+    return launch_b_variant<1, true>(a, plan, b_geometry<true>(a.M), stream, why);
+  }
+  const BGeometry geo = b_geometry<false>(a.M);
   switch (geo.bt / 16) {
     case 1:
-      return launch_b_variant<1>(a, plan, geo, stream, why);
+      return launch_b_variant<1, false>(a, plan, geo, stream, why);
     case 2:
-      return launch_b_variant<2>(a, plan, geo, stream, why);
+      return launch_b_variant<2, false>(a, plan, geo, stream, why);
     case 3:
-      return launch_b_variant<3>(a, plan, geo, stream, why);
+      return launch_b_variant<3, false>(a, plan, geo, stream, why);
     default:
-      return launch_b_variant<4>(a, plan, geo, stream, why);
+      return launch_b_variant<4, false>(a, plan, geo, stream, why);
   }
 }
 

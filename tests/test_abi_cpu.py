@@ -202,18 +202,29 @@ def test_prepack_size_f16s(lib):
 
 
 @pytest.mark.parametrize("M,N,K", [(1, 4096, 4096), (16, 11008, 4096), (16, 4096, 11008),
+                                   (8, 256, 1024), (17, 11008, 4096),
                                    (40, 4096, 4096), (64, 256, 1024), (100, 4096, 4096),
                                    (2048, 11008, 4096), (512, 8192, 28672)])
 def test_gemm_plan_f16s(lib, M, N, K):
-    """One CTA per SM with all tokens (M <= 64) or 64 tokens per tile; a K split
-    only while the tiles leave SMs idle, never past one wave, at most 8 and at
-    most K/128; the smallest split reaching 0.8 CTA per SM with <= 11 K blocks
-    per CTA."""
+    """M <= 16: the two-CTA-per-SM variant (16 tokens per tile), K split as the
+    other decode kernels: the smallest split reaching 0.8 CTA per SM with <= 11
+    K blocks per CTA, never past two CTAs per SM.  Otherwise one CTA per SM with
+    all tokens (M <= 64) or 64 tokens per tile; a K split only while the tiles
+    leave SMs idle, never past one wave, at most 8 and at most K/128; the
+    smallest split reaching 0.8 CTA per SM with <= 11 K blocks per CTA."""
     sms, KB = 148, K // 128
     bn, split, ctas = mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, M, N, K, sms)
+    assert 1 <= split <= min(8, KB)
+    if M <= 16:
+        tiles = N // 128
+        assert bn == 128 and ctas == tiles * split and ctas <= 2 * sms
+        for s in range(1, split):
+            assert not (tiles * s * 5 >= sms * 4 and -(-KB // s) <= 11)
+        assert (ctas * 5 >= sms * 4 and -(-KB // split) <= 11) or split == min(8, KB) or \
+            tiles * (split + 1) > 2 * sms
+        return
     tiles = -(-M // 64) * (N // 128)
     assert bn == 128 and ctas == tiles * split
-    assert 1 <= split <= min(8, KB)
     if split > 1:
         assert ctas <= sms
         # no smaller split already met the occupancy and depth goal
@@ -227,10 +238,14 @@ def test_gemm_plan_f16s(lib, M, N, K):
 
 
 def test_gemm_plan_f16s_examples(lib):
-    # decode N = 11008: 86 tiles, a second wave would be needed for split 2
-    assert mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, 16, 11008, 4096, 148) == (128, 1, 86)
+    # decode N = 11008: 86 tiles x 3 = 258 CTAs (two per SM), 10-11 K blocks each
+    assert mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, 16, 11008, 4096, 148) == (128, 3, 258)
     # decode N = 4096, K = 4096: 32 tiles x 4 = 128 CTAs, 8 K blocks each
     assert mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, 16, 4096, 4096, 148) == (128, 4, 128)
+    # decode K = 11008: 32 tiles x 8 = 256 CTAs, 10-11 K blocks each
+    assert mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, 1, 4096, 11008, 148) == (128, 8, 256)
+    # 17..64 tokens: one CTA per SM; N = 11008 needs a second wave for split 2
+    assert mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, 64, 11008, 4096, 148) == (128, 1, 86)
     # small layer: 4 tiles, split 8 (K = 1024: one K block per CTA)
     assert mq.mixq_gemm_plan(mq.MIXQ_W4G128_F16S, 100, 256, 1024, 148) == (128, 8, 32)
 

@@ -111,7 +111,8 @@ def _oracle_layer(X, W, idx, T, rows=None):
                                          (24, 1024, 512, 16), (40, 2048, 384, 32),
                                          (64, 1024, 640, 64), (100, 512, 256, 4),
                                          (130, 768, 512, 130), (300, 1024, 256, 0),
-                                         (16, 1024, 4096, 32)])
+                                         (16, 1024, 4096, 32), (8, 1024, 28672, 64),
+                                         (16, 4096, 256, 0)])
 def test_layer_within_tolerance(gpu, M, K, N, k_out):
     idx = synth.outlier_channels(K, k_out)
     X = synth.activations(M, K, idx, synth.channel_factors(k_out)) if k_out else \
@@ -121,8 +122,9 @@ def test_layer_within_tolerance(gpu, M, K, N, k_out):
                    f"M{M} K{K} N{N} ko{k_out}")
 
 
-def test_no_token_mixed_and_null_flags(gpu):
-    M, K, N = 48, 2048, 512
+@pytest.mark.parametrize("M", [48, 8])
+def test_no_token_mixed_and_null_flags(gpu, M):
+    K, N = 2048, 512
     idx = synth.outlier_channels(K, 64)
     X = synth.activations(M, K)  # unscaled: no token above T
     W = synth.weights(N, K)
