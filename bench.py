@@ -137,9 +137,9 @@ def quantize_launches(M: int, K: int) -> int:
     """Kernels one mixq_quantize_act call launches: one cluster for decode-sized M
     (at most 16 CTAs of 1024 threads), else a reset pass and the main pass."""
     nvec = K // 8
-    if 0 < M <= 64 and ((nvec <= 512 and (M + 1) // 2 <= 16) or (512 < nvec <= 2048 and M <= 16)):
-        return 1
-    return 2
+    one_cluster = (nvec <= 512 and (M + 3) // 4 <= 16) or \
+        (512 < nvec <= 2048 and M <= 16) or (512 < nvec <= 1536 and (M + 1) // 2 <= 16)
+    return 1 if 0 < M <= 64 and one_cluster else 2
 
 
 def _code_only(text: str) -> str:

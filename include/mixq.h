@@ -147,10 +147,11 @@ mixq_status mixq_prepack_weights(int mode, const void *W, int N, int K, const in
  *                  flags[0] on the device to skip the FP16 slice when no
  *                  token is mixed.
  * K must not exceed 32768 (a token's row is held in registers).
- * For M <= 16 G tokens (G = 2 when K <= 4096, G = 1 when 4096 < K <= 16384)
- * one thread-block cluster of at most 16 CTAs covers the matrix and the call
- * is one kernel; otherwise it is a 1-block reset of bitmap/flags followed by
- * the main pass.
+ * When one thread-block cluster of at most 16 CTAs covers the matrix the call
+ * is one kernel: M <= 64 with K <= 4096 (2 tokens per CTA up to M = 32, 4
+ * above), M <= 16 with K <= 16384 (1 token per CTA), M <= 32 with K <= 12288
+ * (2 tokens per CTA); otherwise it is a 1-block reset of bitmap/flags
+ * followed by the main pass.
  */
 mixq_status mixq_quantize_act(const void *X, int M, int K, int ldx, const int32_t *idx, int K_out,
                               float threshold, int8_t *Xq, float *s_x, void *X_out,

@@ -194,8 +194,9 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   }
 
   // The group's next token is loaded while this one is processed (when the
-  // two rows fit in registers).
-  constexpr bool kPrefetch = VPT <= 8;
+  // two rows fit in registers).  Only the 256-thread grid-stride shapes give
+  // a group a second token; the wide decode shapes launch a group per token.
+  constexpr bool kPrefetch = VPT <= 8 && G * RT == kRowThreads;
   constexpr int kVn = kPrefetch ? VPT : 1;
   auto load_row = [&](int row, uint4 *dst, int count) {
 #pragma unroll
@@ -517,9 +518,17 @@ cudaError_t launch_quantize_act_static(const void *X, int M, int K, int ldx, con
       a.cluster_mode = 1;
       return launch_variant<1, 2, 512, true>(a, (M + 1) / 2, (M + 1) / 2, stream);
     }
+    if (nvec <= 512 && (M + 3) / 4 <= kMaxClusterCtas) {
+      a.cluster_mode = 1;
+      return launch_variant<2, 4, 256, true>(a, (M + 3) / 4, (M + 3) / 4, stream);
+    }
     if (nvec > 512 && nvec <= 2048 && M <= kMaxClusterCtas) {
       a.cluster_mode = 1;
       return launch_variant<2, 1, 1024, true>(a, M, M, stream);
+    }
+    if (nvec > 512 && nvec <= 1536 && (M + 1) / 2 <= kMaxClusterCtas) {
+      a.cluster_mode = 1;
+      return launch_variant<3, 2, 512, true>(a, (M + 1) / 2, (M + 1) / 2, stream);
     }
   }
   const int vpt_need = (nvec + kRowThreads - 1) / kRowThreads;
@@ -580,13 +589,25 @@ cudaError_t launch_quantize_act(const void *X, int M, int K, int ldx, const int3
     // is one token's latency chain, measured: a second token per group adds
     // 2-4 us), all groups in one cluster when that takes at most 16 CTAs (no
     // reset pass, no atomics).
-    if (nvec <= 512 && (M + 1) / 2 <= kMaxClusterCtas) {  // K <= 4096: 2 x 512 threads
+    // K <= 4096: 2 x 512 threads per CTA up to 32 tokens, 4 x 256 up to 64
+    if (nvec <= 512 && (M + 1) / 2 <= kMaxClusterCtas) {
       a.cluster_mode = 1;
       return launch_variant<1, 2, 512>(a, (M + 1) / 2, (M + 1) / 2, stream);
     }
-    if (nvec > 512 && nvec <= 2048 && M <= kMaxClusterCtas) {  // K <= 16384: 1024 threads
+    if (nvec <= 512 && (M + 3) / 4 <= kMaxClusterCtas) {
+      a.cluster_mode = 1;
+      return launch_variant<2, 4, 256>(a, (M + 3) / 4, (M + 3) / 4, stream);
+    }
+    // K <= 16384: 1024 threads per token up to 16 tokens; K <= 12288: 2 x 512
+    // up to 32 (with four 256-thread tokens per CTA, 16 CTAs streaming 64
+    // tokens of K = 11008 measured slower than 64 CTAs and the reset pass)
+    if (nvec > 512 && nvec <= 2048 && M <= kMaxClusterCtas) {
       a.cluster_mode = 1;
       return launch_variant<2, 1, 1024>(a, M, M, stream);
+    }
+    if (nvec > 512 && nvec <= 1536 && (M + 1) / 2 <= kMaxClusterCtas) {
+      a.cluster_mode = 1;
+      return launch_variant<3, 2, 512>(a, (M + 1) / 2, (M + 1) / 2, stream);
     }
   }
   // Otherwise one token per 256-thread CTA at a time (grid-stride over tokens)

@@ -91,7 +91,9 @@ def test_quantize_golden_cases_on_gpu(gpu, gset):
 
 
 @pytest.mark.parametrize("M,K,k_out", [(1, 128, 0), (1, 256, 1), (3, 384, 5), (129, 512, 64),
-                                       (300, 1024, 130), (5, 256, 256), (2, 28672, 64)])
+                                       (300, 1024, 130), (5, 256, 256), (2, 28672, 64),
+                                       (33, 4096, 64), (24, 8192, 64), (64, 11008, 64),
+                                       (48, 12288, 100)])
 def test_quantize_shapes(gpu, M, K, k_out):
     idx = synth.outlier_channels(K, k_out)
     X = synth.activations(M, K, idx, synth.channel_factors(k_out)) if k_out else \
