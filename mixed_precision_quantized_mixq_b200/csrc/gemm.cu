@@ -234,10 +234,12 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
       const uint64_t pol_a = policy_evict_last();
       const uint64_t pol_b = p.b_streamed ? policy_evict_first() : policy_evict_last();
       griddep_wait();
-      const int n_out = (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
-      const int njobs = n_i8 + n_out;
+      // the token tiles of the early stages go out before the flags word is
+      // read: queued behind the weight stream, that read takes microseconds
       for (int j = 0; j < pre; ++j)
         tma_load_2d(a_slot(j), &tm_a, &full[j], (kb_begin + j) * kBlockK, m0, pol_a);
+      const int n_out = (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
+      const int njobs = n_i8 + n_out;
       int issued = pre;
       int s = pre == stages ? 0 : pre;
       uint32_t ph = pre == stages ? 1u : 0u;
@@ -280,12 +282,20 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
       constexpr uint64_t b_step = static_cast<uint64_t>(C::kBStage >> 4);
       uint64_t *const gate = W4 ? ready : full;
       griddep_wait();
-      const int n_out = (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
-      const int njobs = p.debug_stall ? 1 : n_i8 + n_out;
+      // the INT8 jobs first: the flags word (is there an outlier slice) is
+      // read once they are issued, off the path of the first MMAs
+      int njobs = p.debug_stall ? 1 : n_i8;
+      bool counted = p.debug_stall != 0;
       int s = 0, j = 0;
       uint32_t ph = 0;
       uint64_t ad = ad0, bd = bd0;
-      for (; j < njobs; ++j) {
+      for (;; ++j) {
+        if (j == njobs) {
+          if (counted) break;
+          counted = true;
+          njobs += (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
+          if (j == njobs) break;
+        }
         if (!mbar_try_wait(&gate[s], ph) && !mbar_wait(&gate[s], ph, p.wait_limit_ns)) {
           fail(s_err, p.status);
           break;
@@ -331,10 +341,18 @@ __global__ void __launch_bounds__(Cfg<BN, W4, SM>::kThreads, Cfg<BN, W4, SM>::kM
     const int et = threadIdx.x - 128;
     const int row = et % BN;
     const int c0 = W4 ? (et / BN) * kCpt : 0;
-    griddep_wait();
-    const int n_out = (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
-    const int njobs = p.debug_stall ? 0 : n_i8 + n_out;
-    for (int j = 0; j < njobs; ++j) {
+    // the INT8 jobs need nothing from the preceding kernel; the flags word is
+    // read (after waiting for that kernel) once they are done
+    int njobs = p.debug_stall ? 0 : n_i8;
+    bool counted = p.debug_stall != 0;
+    for (int j = 0;; ++j) {
+      if (j == njobs) {
+        if (counted) break;
+        counted = true;
+        griddep_wait();
+        njobs += (outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kOutBlockK : 0;
+        if (j == njobs) break;
+      }
       const int s = j % stages;
       const uint32_t ph = (j / stages) & 1;
       if (!mbar_wait(&full[s], ph, p.wait_limit_ns)) {

@@ -274,10 +274,12 @@ __global__ void __launch_bounds__(kBThreads, BCfg<SM2>::kMinBlocks)
       const uint64_t pol_a = policy_evict_last();
       const uint64_t pol_w = p.w_streamed ? policy_evict_first() : policy_evict_last();
       griddep_wait();
-      const int n_out = (b_outliers_present(p) && rank == 0) ? p.K_out_pad / kBOutK : 0;
-      const int njobs = n_i8 + n_out;
+      // the token tiles of the early stages go out before the flags word is
+      // read: queued behind the weight stream, that read takes microseconds
       for (int j = 0; j < pre; ++j) issue_t(j, j, pol_a);
       s_misc[2] = pre;
+      const int n_out = (b_outliers_present(p) && rank == 0) ? p.K_out_pad / kBOutK : 0;
+      const int njobs = n_i8 + n_out;
       BRing r;
       r.slot = pre == stages ? 0 : pre;
       r.phase = pre == stages ? 1u : 0u;
@@ -309,12 +311,20 @@ __global__ void __launch_bounds__(kBThreads, BCfg<SM2>::kMinBlocks)
       const uint32_t id_i8 = idesc_s8_s32(128, BT);
       const uint32_t id_f16 = idesc_f16_f32(128, BT);
       griddep_wait();
-      const int n_out = (b_outliers_present(p) && rank == 0) ? p.K_out_pad / kBOutK : 0;
-      const int njobs = n_i8 + n_out;
+      // the INT8 jobs first: the flags word (is there an outlier slice) is
+      // read once they are issued, off the path of the first MMAs
+      int njobs = n_i8;
+      bool counted = false;
       BRing r, ra;
       int gi = 0;  // group of this CTA's K range
       bool ok = true;
-      for (int j = 0; j < njobs && ok; ++j) {
+      for (int j = 0; ok; ++j) {
+        if (j == njobs) {
+          if (counted) break;
+          counted = true;
+          njobs += (b_outliers_present(p) && rank == 0) ? p.K_out_pad / kBOutK : 0;
+          if (j == njobs) break;
+        }
         const int s = r.slot;
         if (j < n_i8) {
           if (!mbar_wait(&tfull[s], r.phase, p.wait_limit_ns) ||

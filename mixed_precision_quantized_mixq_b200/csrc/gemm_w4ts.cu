@@ -276,10 +276,12 @@ __global__ void __launch_bounds__(kTsThreads, TsCfg<SM>::kMinBlocks)
       const uint64_t pol_a = policy_evict_last();
       const uint64_t pol_w = p.w_streamed ? policy_evict_first() : policy_evict_last();
       griddep_wait();
-      const int n_out = (ts_outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kTsOutK : 0;
-      const int njobs = n_i8 + n_out;
+      // the token tiles of the early stages go out before the flags word is
+      // read: queued behind the weight stream, that read takes microseconds
       for (int j = 0; j < pre; ++j) issue_t(j, j, pol_a);
       s_misc[2] = pre;
+      const int n_out = (ts_outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kTsOutK : 0;
+      const int njobs = n_i8 + n_out;
       RingPos r;  // position of job j (no division in the loop)
       r.slot = pre == stages ? 0 : pre;
       r.phase = pre == stages ? 1u : 0u;
@@ -314,10 +316,18 @@ __global__ void __launch_bounds__(kTsThreads, TsCfg<SM>::kMinBlocks)
       const uint64_t bd0 = sw128_kmajor_desc(smem_u32(stage(0) + p.w_slot));
       const uint64_t st_step = static_cast<uint64_t>(p.stage_bytes >> 4);
       griddep_wait();
-      const int n_out = (ts_outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kTsOutK : 0;
-      const int njobs = n_i8 + n_out;
+      // the INT8 jobs first: the flags word (is there an outlier slice) is
+      // read once they are issued, off the path of the first MMAs
+      int njobs = n_i8;
+      bool counted = false;
       RingPos r, ra;
-      for (int j = 0; j < njobs; ++j) {
+      for (int j = 0;; ++j) {
+        if (j == njobs) {
+          if (counted) break;
+          counted = true;
+          njobs += (ts_outliers_present(p, RAW) && rank == 0) ? p.K_out_pad / kTsOutK : 0;
+          if (j == njobs) break;
+        }
         const int s = r.slot;
         if (j < n_i8) {
           if (!mbar_wait(&tfull[s], r.phase, p.wait_limit_ns) ||
