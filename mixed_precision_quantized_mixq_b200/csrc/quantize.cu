@@ -84,6 +84,12 @@ __device__ __forceinline__ int warp_sum(int v) {
   return v;
 }
 
+__device__ __forceinline__ __half2 u32_as_half2(uint32_t w) {
+  __half2 h;
+  memcpy(&h, &w, sizeof h);
+  return h;
+}
+
 // clamp(rint(x * inv), -127, 127): one IEEE fp32 multiply, round half to even.
 __device__ __forceinline__ uint32_t code8(float x, float inv) {
   int q = __float2int_rn(__fmul_rn(x, inv));
@@ -125,9 +131,17 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   uint32_t *s_mask = qsm;               // outlier channel bitset
   uint32_t *s_det = qsm + words;        // channels with |x| > T seen by this CTA
   uint32_t *s_rank = qsm + 2 * words;   // outlier channels in words before w
+  // the group's X_out row of a mixed token, written out with 16-byte stores
+  // (the padding columns stay zero: they are cleared once and never written)
+  __half *s_xo = reinterpret_cast<__half *>(qsm + 3 * words) + (threadIdx.x / RT) * a.K_out_pad;
   __shared__ float s_red[G][2][kRowWarps];
   __shared__ int s_bad, s_last, s_part[2], s_cnt[G * kRowWarps];
   __shared__ uint32_t s_mixed_total;  // cluster mode: rank 0 accumulates every CTA's count
+  // Lane masks of an 8-channel vector by its outlier bits b (bit e = channel
+  // e is in idx): s_keep[b] word p keeps the magnitude bits (0x7FFF) of the
+  // non-outlier halves of pair p, s_bkeep[b] keeps their code bytes.
+  __shared__ uint4 s_keep[256];
+  __shared__ uint2 s_bkeep[256];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = tid / RT, gt = tid % RT, gw = gt >> 5;
@@ -146,6 +160,18 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   for (int w = tid; w < words; w += blockDim.x) {
     s_mask[w] = 0u;
     s_det[w] = 0u;
+  }
+  for (int j = tid % RT; j < a.K_out_pad; j += RT) s_xo[j] = __ushort_as_half(0);
+  for (int b = tid; b < 256; b += blockDim.x) {
+    uint32_t hk[4], bk[2] = {0u, 0u};
+#pragma unroll
+    for (int p = 0; p < 4; ++p)
+      hk[p] = (((b >> (2 * p)) & 1) ? 0u : 0x7FFFu) | (((b >> (2 * p + 1)) & 1) ? 0u : 0x7FFF0000u);
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+      if (!((b >> e) & 1)) bk[e >> 2] |= 0xFFu << (8 * (e & 3));
+    s_keep[b] = make_uint4(hk[0], hk[1], hk[2], hk[3]);
+    s_bkeep[b] = make_uint2(bk[0], bk[1]);
   }
   if (tid == 0) {
     s_bad = 0;
@@ -181,6 +207,7 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
     }
   }
   __syncthreads();
+  const __half t_half = __float2half_rd(a.T);  // |x| > T  <=>  |x| > t_half for fp16 |x|
   griddep_wait();
   if (tid == 0 && s_bad) record_error(a.status, kErrInvalidArg);
   int m = blockIdx.x * G + g;
@@ -209,6 +236,9 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
     }
   };
   int mixed_rows = 0;
+  uint32_t det_acc[VPT];  // detection bits of the thread's vectors over its tokens
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) det_acc[i] = 0u;
   for (; m < a.M; m += row_stride) {
     uint4 vn[kVn];
     if (kPrefetch) load_row(m + row_stride, vn, kVn);
@@ -261,41 +291,55 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
         if (xn_row && vi < nvec) reinterpret_cast<uint4 *>(xn_row)[vi] = v[i];
       }
     }
-    float aI = 0.f, aN = 0.f;
+    // |x| over all channels and over the non-outlier ones, in fp16 (abs and
+    // max are exact there, and max skips NaN like fmaxf), two lanes at a time;
+    // the detection bits only for vectors whose largest |x| is above T
+    // (|x| > T for an fp16 |x| exactly when |x| > T rounded down to fp16)
+    __half2 mA = __float2half2_rn(0.f), mN = mA;
 #pragma unroll
     for (int i = 0; i < VPT; ++i) {
       const int vi = gt + i * RT;
       const int k0 = vi << 3;
       const uint32_t mb = vi < nvec ? (s_mask[k0 >> 5] >> (k0 & 31)) & 0xFFu : 0u;
-      const __half2 *h = reinterpret_cast<const __half2 *>(&v[i]);
-      uint32_t det = 0;
+      const uint4 kp = s_keep[mb];
+      const uint32_t hw[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      const uint32_t kw[4] = {kp.x, kp.y, kp.z, kp.w};
+      __half2 vm = __float2half2_rn(0.f);
 #pragma unroll
       for (int e2 = 0; e2 < 4; ++e2) {
-        const float2 f = __half22float2(h[e2]);
-        const float a0 = fabsf(f.x), a1 = fabsf(f.y);
-        if ((mb >> (2 * e2)) & 1u) aI = fmaxf(aI, a0); else aN = fmaxf(aN, a0);
-        if ((mb >> (2 * e2 + 1)) & 1u) aI = fmaxf(aI, a1); else aN = fmaxf(aN, a1);
-        det |= (a0 > a.T ? 1u : 0u) << (2 * e2);
-        det |= (a1 > a.T ? 1u : 0u) << (2 * e2 + 1);
+        vm = __hmax2(vm, u32_as_half2(hw[e2] & 0x7FFF7FFFu));
+        mN = __hmax2(mN, u32_as_half2(hw[e2] & kw[e2]));
       }
-      if (det) atomicOr(&s_det[k0 >> 5], det << (k0 & 31));
+      mA = __hmax2(mA, vm);
+      if (__hgt(__hmax(__low2half(vm), __high2half(vm)), t_half)) {
+        uint32_t det = 0;
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2) {
+          const __half2 ab = u32_as_half2(hw[e2] & 0x7FFF7FFFu);
+          det |= (__hgt(__low2half(ab), t_half) ? 1u : 0u) << (2 * e2);
+          det |= (__hgt(__high2half(ab), t_half) ? 1u : 0u) << (2 * e2 + 1);
+        }
+        det_acc[i] |= det;
+      }
     }
-    aI = warp_max(aI);
+    float aA = fmaxf(__low2float(mA), __high2float(mA));
+    float aN = fmaxf(__low2float(mN), __high2float(mN));
+    aA = warp_max(aA);
     aN = warp_max(aN);
     if (lane == 0) {
-      s_red[g][0][gw] = aI;
+      s_red[g][0][gw] = aA;
       s_red[g][1][gw] = aN;
     }
     named_barrier(1 + g, RT);
-    float rI = s_red[g][0][0], rN = s_red[g][1][0];
+    float rA = s_red[g][0][0], rN = s_red[g][1][0];
 #pragma unroll
     for (int w = 1; w < kRowWarps; ++w) {
-      rI = fmaxf(rI, s_red[g][0][w]);
+      rA = fmaxf(rA, s_red[g][0][w]);
       rN = fmaxf(rN, s_red[g][1][w]);
     }
     named_barrier(1 + g, RT);  // s_red is rewritten by the group's next token
 
-    const float amax = fmaxf(rI, rN);
+    const float amax = rA;
     const bool mixed = a.K_out > 0 && amax > a.T;
     const float am = mixed ? rN : amax;
     const float inv = am > 0.f ? __fdiv_rn(127.f, am) : 0.f;
@@ -314,16 +358,22 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
       const uint32_t word = s_mask[k0 >> 5];
       const uint32_t mb = mixed ? (word >> (k0 & 31)) & 0xFFu : 0u;
       const __half2 *h = reinterpret_cast<const __half2 *>(&v[i]);
-      uint32_t lo = 0, hi = 0;
+      uint32_t q[8];
 #pragma unroll
       for (int e2 = 0; e2 < 4; ++e2) {
         const float2 f = __half22float2(h[e2]);
-        const uint32_t q0 = ((mb >> (2 * e2)) & 1u) ? 0u : code8(f.x, inv);
-        const uint32_t q1 = ((mb >> (2 * e2 + 1)) & 1u) ? 0u : code8(f.y, inv);
-        const uint32_t pair = q0 | (q1 << 8);
-        if (e2 < 2) lo |= pair << (16 * e2);
-        else hi |= pair << (16 * (e2 - 2));
+        q[2 * e2] = code8(f.x, inv);
+        q[2 * e2 + 1] = code8(f.y, inv);
       }
+      // low bytes packed in channel order; the outlier channels of a mixed
+      // token are zero
+      const uint2 bk = s_bkeep[mb];
+      const uint32_t lo =
+          __byte_perm(__byte_perm(q[0], q[1], 0x0040u), __byte_perm(q[2], q[3], 0x0040u), 0x5410u) &
+          bk.x;
+      const uint32_t hi =
+          __byte_perm(__byte_perm(q[4], q[5], 0x0040u), __byte_perm(q[6], q[7], 0x0040u), 0x5410u) &
+          bk.y;
       qr[vi] = make_uint2(lo, hi);
       if (mb) {  // outlier channels of a mixed token -> their X_out columns
         const int base = static_cast<int>(s_rank[k0 >> 5]) +
@@ -333,15 +383,17 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
           if ((mb >> e) & 1u) {
-            orow[j] = __ushort_as_half(hs[e]);
+            s_xo[j] = __ushort_as_half(hs[e]);
             ++j;
           }
         }
       }
     }
-    // every other X_out column of this token is zero
-    for (int j = gt; j < a.K_out_pad; j += RT)
-      if (!mixed || j >= a.K_out) orow[j] = __ushort_as_half(0);
+    // the token's X_out row: its outlier channels (mixed) or zeros
+    if (mixed) named_barrier(1 + g, RT);  // the group's columns are in s_xo
+    for (int j = gt; j < a.K_out_pad / 8; j += RT)
+      reinterpret_cast<uint4 *>(orow)[j] =
+          mixed ? reinterpret_cast<const uint4 *>(s_xo)[j] : make_uint4(0u, 0u, 0u, 0u);
     if (kPrefetch) {
 #pragma unroll
       for (int i = 0; i < kVn; ++i) v[i] = vn[i];
@@ -351,6 +403,11 @@ __global__ void __launch_bounds__(RT *G) quantize_act_kernel(const QArgs a) {
   }
 
   // ------------------------------------------- matrix-wide bitmap and flags
+#pragma unroll
+  for (int i = 0; i < VPT; ++i) {
+    const int k0 = (gt + i * RT) << 3;
+    if (det_acc[i]) atomicOr(&s_det[k0 >> 5], det_acc[i] << (k0 & 31));
+  }
   if (lane == 0) s_cnt[warp] = 0;
   __syncwarp();
   if (gt == 0) s_cnt[warp] = mixed_rows;
@@ -436,7 +493,8 @@ cudaError_t launch_variant(const QArgs &a, int grid, int cluster, cudaStream_t s
     kernel = quantize_act_kernel<VPT, G, RT, false, true>;
   else
     kernel = a.gamma ? quantize_act_kernel<VPT, G, RT, true> : quantize_act_kernel<VPT, G, RT, false>;
-  const size_t smem = sizeof(uint32_t) * 3 * (a.K / 32);
+  // outlier bitset, detection words, rank prefix; one X_out row per group
+  const size_t smem = sizeof(uint32_t) * 3 * (a.K / 32) + sizeof(__half) * G * a.K_out_pad;
   cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem < 48 * 1024 ? 48 * 1024 : smem));
   if (e == cudaSuccess && cluster > 8)

@@ -132,6 +132,33 @@ def test_bad_idx_reported_on_device(gpu):
     assert int(status.item()) == 1
 
 
+@pytest.mark.parametrize("T", [6.0, 6.001, 5.9990234375, 0.3, 1e5])
+@pytest.mark.parametrize("M,K", [(3, 512), (40, 2048), (300, 4096)])
+def test_quantize_threshold_between_fp16_values(gpu, T, M, K):
+    """The outlier test |x| > T with T not an fp16 value: activations placed on
+    the fp16 neighbours of T (and their negatives) in outlier and ordinary
+    channels; codes, scales, X_out, bitmap and flags bit for bit."""
+    rng = np.random.default_rng(int(T * 1000) % 97 + M)
+    X = (rng.standard_normal((M, K)) * 0.3).astype(np.float16)
+    t = np.float16(T) if np.isfinite(np.float16(T)) else np.float16(65504)
+    below = t if float(t) <= T else np.nextafter(t, np.float16(-np.inf))
+    with np.errstate(over="ignore"):
+        neigh = [below, np.nextafter(below, np.float16(np.inf)),
+                 np.nextafter(below, np.float16(-np.inf))]
+    neigh = [n if np.isfinite(n) else np.float16(65504) for n in neigh]
+    idx = synth.outlier_channels(K, 16)
+    cols = [int(idx[1]), int(idx[5]), 7, 300, K - 1]
+    for j, c in enumerate(cols):
+        for r in range(0, M, 3):
+            v = neigh[(j + r) % 3]
+            X[r, c] = v if (r + j) % 2 == 0 else -v
+    W = synth.weights(128, K)
+    g = gpu.layer(X, W, idx, "w8", T)
+    o = oracle_layer(X, W, idx, "w8", T)
+    assert g["status"] == 0
+    _assert_quant_equal(g, o, f"T={T} M{M} K{K}")
+
+
 # ---------------------------------------------------------- INT32 mainloop
 @functools.lru_cache(maxsize=None)
 def _packed_random(N, K, mode_i):
