@@ -35,9 +35,9 @@
 //   warps 2..9      epilogue: warp w reads TMEM lanes 32(w%4).. (weight rows),
 //                   half of the 256 token columns each
 //   warps 10..17    expansion: thread = weight row = TMEM lane; warps 10..13
-//                   take the first K block of every job, 14..17 the second
-//                   (storing a K block to TMEM is the slow step, so two warps
-//                   per lane group keep two stores in flight)
+//                   take the even jobs, 14..17 the odd ones, both K blocks
+//                   each (a TMEM store completes behind the MMAs in flight,
+//                   so two groups keep two jobs' stores in flight)
 // Outlier jobs (64 channels each) carry a W_out tile (A) and an X_out tile (B),
 // both by TMA to the leader's barrier; the outlier product accumulates onto
 // the accumulator after the epilogue has converted it in place to FP32, as in
@@ -57,6 +57,7 @@ namespace {
 constexpr int kQThreads = 576;  // 0 producer, 1 MMA/TMEM, 2..9 epilogue, 10..17 expansion
 constexpr int kQEpiWarps = 8;
 constexpr int kQExpWarps = 8;
+constexpr int kQGroupWarps = 4;  // expansion warps per job (two groups take alternate jobs)
 constexpr int kQBT = 256;                     // tokens per pair tile (MMA N)
 constexpr int kQHalf = kQBT / 2;              // token rows per CTA
 constexpr int kQCodes = 128 * (kBlockK / 2);  // 8 KB of codes per 128 x 128 block
@@ -72,6 +73,10 @@ constexpr int kQTmemCols = 512;
 constexpr int kQACol = kQBT;  // A ring after the accumulator
 constexpr int kQAStages = 4;  // 64 columns each
 static_assert(kQACol + kQAStages * 32 * kQKbJob <= kQTmemCols, "tensor memory");
+// job n uses shared-memory slot n % 4 and (INT8 jobs) A stage n % 4, and is
+// expanded by group n % 2: every slot and stage belongs to one group, whose
+// barrier phases it therefore sees one by one
+static_assert(kQAStages == kQStages && kQStages % 2 == 0, "slot and stage share the job index");
 static_assert(kQWSlot % 1024 == 0 && kQStage % 1024 == 0, "swizzle atoms stay aligned");
 static_assert(kQOutTile <= kQWSlot, "outlier W_out tile fits the weight slot");
 
@@ -200,10 +205,10 @@ __global__ void __launch_bounds__(kQThreads, 1)
     for (int i = 0; i < kQStages; ++i) {
       mbar_init(&wfull[i], 1);
       mbar_init(&tfull[i], 1);
-      mbar_init(&sempty[i], kQExpWarps + 1);
+      mbar_init(&sempty[i], kQGroupWarps + 1);
     }
     for (int a = 0; a < kQAStages; ++a) {
-      mbar_init(&afull[a], 2 * kQExpWarps);
+      mbar_init(&afull[a], 2 * kQGroupWarps);
       mbar_init(&aempty[a], 1);
     }
     mbar_init(acc_full, 1);
@@ -291,7 +296,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                            256 * tn + 128 * static_cast<int>(rank), pol);
           tma_load_2d_pair(tok, &tm_xo, bar, j * 64, row_t, pol);
           mbar_arrive(&wfull[slot]);  // every use of a slot completes one phase
-          mbar_arrive_cnt(&sempty[slot], kQExpWarps);
+          mbar_arrive_cnt(&sempty[slot], kQGroupWarps);
         }
         ++n;
         if (++slot == kQStages) {
@@ -312,11 +317,12 @@ __global__ void __launch_bounds__(kQThreads, 1)
       constexpr uint64_t kStageD = kQStage >> 4, kTokD = kQTok >> 4;
       griddep_wait();
       const int chunks_o = q_outliers(p, RAW) ? p.K_out_pad / 64 : 0;
-      int slot = 0, n = 0, as = 0;
-      uint32_t phase = 0, aph = 0;
+      int slot = 0, n = 0;
+      uint32_t phase = 0, aph = 0;  // aph: phase bit of each A stage (INT8 uses only)
       bool ok = true;
       q_for_each_job(iters, jobs8, KB, chunks_o, [&](int kind, int it, int j, int nkb) {
         const uint32_t use = static_cast<uint32_t>(it);
+        const int as = slot;
         if (kind == 0 && j == 0 && it >= 1) {
           // the previous tile's accumulator has been drained by both CTAs
           if (!mbar_wait_sleep(tmem_empty, (use - 1) & 1, p.wait_limit_ns)) return ok = false;
@@ -330,7 +336,8 @@ __global__ void __launch_bounds__(kQThreads, 1)
           return ok = false;
         const uint32_t d = tmem_base;
         if (kind == 0) {
-          if (!mbar_try_wait(&afull[as], aph) && !mbar_wait(&afull[as], aph, p.wait_limit_ns))
+          const uint32_t ap = (aph >> as) & 1u;
+          if (!mbar_try_wait(&afull[as], ap) && !mbar_wait(&afull[as], ap, p.wait_limit_ns))
             return ok = false;
           tc_fence_after();
           const uint64_t bd = bd0 + slot * kStageD;
@@ -342,10 +349,7 @@ __global__ void __launch_bounds__(kQThreads, 1)
                              (j > 0 || kk > 0 || k > 0) ? 1u : 0u);
           }
           mma_commit_pair(&aempty[as], 3);
-          if (++as == kQAStages) {
-            as = 0;
-            aph ^= 1u;
-          }
+          aph ^= 1u << as;
         } else {
           tc_fence_after();
           const uint64_t ad = od0 + slot * kStageD, bd = bd0 + slot * kStageD;
@@ -371,12 +375,16 @@ __global__ void __launch_bounds__(kQThreads, 1)
     }
   } else if (warp >= 10) {
     // ------------------------------------------- 4-bit -> INT8 expansion
+    // Two groups of four warps take alternate jobs (storing to TMEM waits
+    // behind the MMAs in flight, so a group keeps one job's store in flight
+    // while the other expands the next job); a warp expands both K blocks of
+    // its job for its 32 weight rows.
     const int row = (warp & 3) * 32 + lane;  // weight row of this CTA's 128 = TMEM lane
-    const int sub = (warp - 10) >> 2;        // K block of each job this warp expands
+    const int grp = (warp - 10) >> 2;        // jobs n with n % 2 == grp
     const uint32_t lane_addr = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t afull_w = afull_l;
-    int slot = 0, as = 0;
-    uint32_t phase = 0, aph = 0;
+    int slot = 0, n = 0;
+    uint32_t phase = 0, aph = 0;  // aph: phase bit of each A stage (INT8 uses only)
     bool ok = true;
     if (iters > 0) {
       griddep_wait();
@@ -384,34 +392,34 @@ __global__ void __launch_bounds__(kQThreads, 1)
       q_for_each_job(iters, jobs8, KB, chunks_o, [&](int kind, int it, int j, int nkb) {
         (void)it;
         (void)j;
-        if (kind == 0) {
-          if (!q_warp_wait(&wfull[slot], phase, p.wait_limit_ns)) return ok = false;
-          const uint8_t *sp = stage(slot);
-          const bool mine = sub < nkb;  // a job's second K block may not exist
-          uint32_t wv[32];
-          if (mine) q_expand_block(sp + sub * kQCodes, sp + kQKbJob * kQCodes + sub * kQGrp, row, wv);
-          __syncwarp();
-          if (lane == 0) mbar_arrive(&sempty[slot]);  // codes read
-          // A stage `as` was last read by the MMAs kQAStages jobs ago
-          if (!q_warp_wait(&aempty[as], aph ^ 1, p.wait_limit_ns)) return ok = false;
-          tc_fence_after();
-          if (mine) {
-            tmem_st32(t_a + lane_addr + static_cast<uint32_t>(as * 32 * kQKbJob + sub * 32), wv);
-            tmem_st_wait();
-          }
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive_cluster(afull_w + 8u * as);
-          if (++as == kQAStages) {
-            as = 0;
-            aph ^= 1u;
-          }
-        } else {
+        if ((n & 1) == grp) {
           // an outlier job's stage carries no codes, but its phase of wfull is
-          // waited for all the same: a warp that skipped it could run two
+          // waited for all the same: a group that skipped it could run two
           // phases ahead of the barrier, where a parity wait cannot tell them apart
           if (!q_warp_wait(&wfull[slot], phase, p.wait_limit_ns)) return ok = false;
+          if (kind == 0) {
+            const int as = slot;
+            const uint8_t *sp = stage(slot);
+            uint32_t wv0[32], wv1[32];
+            q_expand_block(sp, sp + kQKbJob * kQCodes, row, wv0);
+            if (nkb > 1) q_expand_block(sp + kQCodes, sp + kQKbJob * kQCodes + kQGrp, row, wv1);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sempty[slot]);  // codes read
+            // A stage `as` was last read by the MMAs of this group's job kQAStages jobs ago
+            if (!q_warp_wait(&aempty[as], ((aph >> as) & 1u) ^ 1u, p.wait_limit_ns))
+              return ok = false;
+            tc_fence_after();
+            const uint32_t ta = t_a + lane_addr + static_cast<uint32_t>(as * 32 * kQKbJob);
+            tmem_st32(ta, wv0);
+            if (nkb > 1) tmem_st32(ta + 32, wv1);
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(afull_w + 8u * as);
+            aph ^= 1u << as;
+          }
         }
+        ++n;
         if (++slot == kQStages) {
           slot = 0;
           phase ^= 1u;
