@@ -482,33 +482,47 @@ __global__ void __launch_bounds__(kQThreads, 1)
         }
         tc_fence_after();
       }
+      // two 32-token chunks per TMEM round trip; the accumulator is released
+      // after the last load, so the next tile's MMAs overlap the last stores
 #pragma unroll 1
-      for (int c = 0; c < kQHalf / 32; ++c) {
+      for (int c = 0; c < kQHalf / 32; c += 2) {
         const int col = kQHalf * h + 32 * c;
-        uint32_t v[32];
-        tmem_ld32(d + col, v);
+        uint32_t v[2][32];
+        tmem_ld32(d + col, v[0]);
+        tmem_ld32(d + col + 32, v[1]);
         tmem_ld_wait();
+        if (c + 2 == kQHalf / 32) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster(tmem_empty_l);
+        }
         if (n >= p.N) continue;
 #pragma unroll
-        for (int e = 0; e < 32; ++e) {
-          const int m = m_base + col + e;
-          if (m >= p.M) break;
+        for (int hh = 0; hh < 2; ++hh) {
+          const int m0c = m_base + col + 32 * hh;
+          const int mcount = min(32, p.M - m0c);
+          if (mcount <= 0) break;
+          const size_t off0 = static_cast<size_t>(m0c) * p.ldy + n;
           if (RAW) {
-            static_cast<int32_t *>(p.Y)[static_cast<size_t>(m) * p.ldy + n] =
-                static_cast<int32_t>(v[e]);
+            int32_t *yp = static_cast<int32_t *>(p.Y) + off0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (e < mcount) yp[static_cast<size_t>(e) * p.ldy] = static_cast<int32_t>(v[hh][e]);
           } else {
-            const float y = chunks_o > 0
-                                ? __uint_as_float(v[e])
-                                : __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(v[e])),
-                                                      sx[col + e]),
-                                            sw);
-            static_cast<__half *>(p.Y)[static_cast<size_t>(m) * p.ldy + n] = __float2half_rn(y);
+            __half *yp = static_cast<__half *>(p.Y) + off0;
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (e >= mcount) break;
+              const float y =
+                  chunks_o > 0 ? __uint_as_float(v[hh][e])
+                               : __fmul_rn(__fmul_rn(static_cast<float>(static_cast<int>(v[hh][e])),
+                                                     sx[col + 32 * hh + e]),
+                                           sw);
+              yp[static_cast<size_t>(e) * p.ldy] = __float2half_rn(y);
+            }
           }
         }
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_cluster(tmem_empty_l);
     }
     if (!ok) q_fail(s_err, p.status);
   }
