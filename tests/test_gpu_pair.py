@@ -111,8 +111,12 @@ def test_pair_layer_no_token_mixed_and_null_flags(gpu):
 # ------------------------------------------------------------ 4-bit weights
 @pytest.mark.parametrize("M,N,K", [(256, 256, 128), (512, 512, 1024), (300, 384, 512),
                                    (1000, 1280, 2048), (2048, 4096, 1024), (257, 4992, 256),
-                                   (200, 256, 384)])
+                                   (200, 256, 384), (2048, 8192, 640), (2304, 8064, 384)])
 def test_pair_w4_int32_bit_exact(gpu, M, N, K):
+    # (2048, 8192, 640): three jobs per tile (an odd count) over several tiles
+    # per pair, so consecutive tiles start on jobs of either expansion group
+    # and on any shared-memory slot; (2304, 8064, 384): a one-block last job,
+    # and N % 256 == 128 (the second CTA's rows of the last column tile absent)
     torch, mq = gpu.torch, gpu.mq
     W = synth.weights(N, K, seed=M + N + 1)
     w = mq.prepack(gpu.dev(W), gpu.dev(np.zeros(0, np.int32)), mq.MIXQ_W4G128)
@@ -137,8 +141,11 @@ def test_pair_w4_int32_matches_the_tensor_memory_kernel(gpu):
 
 @pytest.mark.parametrize("M,N,K,k_out", [(2048, 5120, 1024, 64), (2304, 4992, 2048, 256),
                                          (2048, 5120, 1024, 0), (2048, 11008, 4096, 128),
-                                         (2100, 640, 384, 32), (4096, 4096, 4096, 256)])
+                                         (2100, 640, 384, 32), (4096, 4096, 4096, 256),
+                                         (2048, 8192, 640, 128), (2560, 6144, 1152, 128)])
 def test_pair_w4_layer_within_tolerance(gpu, M, N, K, k_out):
+    # the last two: odd job counts per tile (3 INT8 + 2 outlier jobs; 5 + 2)
+    # over several tiles per pair
     mq = gpu.mq
     assert mq.mixq_gemm_plan(mq.MIXQ_W4G128, M, N, K)[0] == 256
     idx = synth.outlier_channels(K, k_out)
